@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Verify-step benchmark: verify-steps/s and accepted tokens/s on B200.
+
+One step = the whole verify hot path for one batch: sv_verify_attention for
+every layer of the named model shape (each layer with its own KV pool, so no
+layer reads another's bytes from L2) followed by one sv_accept over the
+vocabulary. The timed work per step (several GB of KV) is far larger than the
+126 MB L2, so no flush is needed between steps.
+
+Default workload: Qwen2.5-7B-shaped layer in the long-tail phase (B=8 active
+sequences, 28 q heads / 4 kv heads, D=128, contexts uniform 4k-16k, gamma=4,
+vocab 152064, T=1), 28 layers.
+
+--impl reference times the fp64 CPU oracle on the host cores instead (the
+baseline arm: the pages ship no runnable implementation of this path).
+Multi-GPU (torchrun): every rank runs its own replica of the workload
+(sequences are independent; no data-path collective); value = all ranks'
+steps / max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from speculative_decoding_rl_b200 import workloads as W  # noqa: E402
+
+METRIC = "verify-steps/s & accepted tok/s at 1 B200; KV+logit HBM GB/s as % of peak"
+UNIT = "verify-steps/s"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qwen7b_longtail")
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "speculative_decoding_rl_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per attention launch from a committed ncu summary, if it
+    matches the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_hash") != kernel_source_hash() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_call")
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w: W.Workload, a0, acc, layers: int, budget_s: float, seed: int = 0):
+    """Time the oracle on a bounded sample and scale to verify-steps/s.
+
+    Attention: whole query-row sets of a few (sequence, KV head) units, scaled
+    by the ratio of total to sampled (rows x visible keys) work. Accept: the
+    whole batch (every sequence), timed once."""
+    import oracle
+    B, N, Hq, Hkv = a0.num_seqs, a0.num_q_rows, a0.num_q_heads, a0.num_kv_heads
+    G = Hq // Hkv
+    lens = a0.ctx_lens.numpy()
+    total_work = float(lens.sum()) * N * Hq
+    rng = np.random.default_rng(seed)
+    units = rng.permutation(B * Hkv)
+    t_attn, work = 0.0, 0.0
+    t0 = time.perf_counter()
+    for u in units:
+        b, h = divmod(int(u), Hkv)
+        rows = np.array([[b, i, h * G + g] for i in range(N) for g in range(G)], dtype=np.int32)
+        s = time.perf_counter()
+        oracle.attention_rows(a0, rows)
+        t_attn += time.perf_counter() - s
+        work += float(lens[b]) * N * G
+        if time.perf_counter() - t0 > budget_s * 0.7:
+            break
+    s = time.perf_counter()
+    oracle.accept(acc.target_logits, acc.draft_probs, acc.draft_tokens, acc.temperature, seed,
+                  parents=acc.tree_parents)
+    t_acc = time.perf_counter() - s
+    t_attn_layer = t_attn * total_work / work
+    step = layers * t_attn_layer + t_acc
+    sample = (f"oracle attention on {work / (N * G):.0f} of {lens.sum() * Hkv} (sequence, kv-head) keys "
+              f"({100 * work / total_work:.1f}% of one layer, scaled by work to {layers} layers) "
+              f"+ oracle accept on all {B} sequences; single-threaded fp64")
+    return 1.0 / step, t_attn_layer, t_acc, sample
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    w = W.workload(args.workload)
+    layers = args.layers or w.num_layers
+    a0 = W.build_attention(w)
+    acc = W.build_accept(w)
+    budget = max(2.0, 120.0 / max(1, args.steps + args.warmup))
+    vals = []
+    for k in range(args.warmup + args.steps):
+        v, _, _, sample = oracle_sample(w, a0, acc, layers, budget, seed=k)
+        if k >= args.warmup:
+            vals.append(v)
+    value = statistics.median(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / value,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "layers": layers},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import speculative_decoding_rl_b200 as sv
+    from speculative_decoding_rl_b200.session import AcceptCall, AttentionCall
+
+    dev = torch.device("cuda", local)
+    w = W.workload(args.workload)
+    layers = args.layers or w.num_layers
+    a0 = W.build_attention(w)
+    acc_in = W.build_accept(w)
+    B, N, Hq, D = a0.num_seqs, a0.num_q_rows, a0.num_q_heads, a0.head_dim
+
+    # Layer 0 from the seeded CPU generator; layers 1.. get their own pools and
+    # queries drawn on the device (same sequences and page tables).
+    calls = [AttentionCall(a0, device=str(dev))]
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + rank)
+    for _ in range(1, layers):
+        c = AttentionCall.__new__(AttentionCall)
+        c.inputs = a0
+        c.desc = calls[0].desc
+        c.block_table, c.ctx_lens, c.mask = calls[0].block_table, calls[0].ctx_lens, calls[0].mask
+        c.k_pool = torch.randn(a0.k_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
+        c.v_pool = torch.randn(a0.v_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
+        c.q = torch.randn(a0.q.shape, generator=g, device=dev, dtype=torch.bfloat16)
+        c.out = torch.empty_like(c.q)
+        c.status = None
+        c.ws_bytes, c.workspace = calls[0].ws_bytes, calls[0].workspace
+        c.kv = sv.SvPagedKV(c.k_pool.data_ptr(), c.v_pool.data_ptr())
+        calls.append(c)
+    acc = AcceptCall(acc_in, device=str(dev), seed=0)
+    stream = torch.cuda.current_stream(dev)
+
+    K, Wm = args.steps, args.warmup
+    lens_out = torch.zeros((Wm + K, B), dtype=torch.int32, device=dev)
+
+    def step(k, ev_pairs=None):
+        for li, c in enumerate(calls):
+            if ev_pairs is not None:
+                ev_pairs[li][0].record(stream)
+            c.run(stream)
+            if ev_pairs is not None:
+                ev_pairs[li][1].record(stream)
+        acc.seed = k
+        acc.accept_len = lens_out[k]
+        acc.run(stream)
+
+    # parity spot check before timing: sampled attention rows of layer 0 and the accept
+    import oracle
+    step(0)
+    torch.cuda.synchronize()
+    rows = np.stack([np.arange(16) % B, (np.arange(16) * 3) % N, (np.arange(16) * 7) % Hq], 1).astype(np.int32)
+    ref = oracle.attention_rows(a0, rows)
+    got = calls[0].out.float().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
+    parity_attn = float(np.abs(got - ref).max())
+    o = oracle.accept(acc_in.target_logits, acc_in.draft_probs, acc_in.draft_tokens, acc_in.temperature, 0,
+                      parents=acc_in.tree_parents)
+    ok = (o.tie_depth >= 0) | (o.tie_draw > 0) | ((lens_out[0].cpu().numpy() == o.accept_len)
+                                                 & (acc.next_token.cpu().numpy() == o.next_token))
+    parity = {"attn_max_abs_sampled": parity_attn, "accept_seqs_matching": int(ok.sum()), "accept_seqs": B}
+
+    for k in range(1, Wm):
+        step(k)
+    torch.cuda.synchronize()
+    barrier(world)
+
+    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(layers)]
+    per_call = []
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        torch.cuda.synchronize()
+        barrier(world)
+        start.record(stream)
+        for k in range(Wm, Wm + K):
+            step(k, ev if k == Wm + K - 1 else None)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed = start.elapsed_time(end) / 1e3
+    per_call = [a.elapsed_time(b) / 1e3 for a, b in ev]
+    # per-call timing on a separate pass (events around every attention call, all steps)
+    ev_all = []
+    torch.cuda.synchronize()
+    for k in range(Wm, Wm + min(K, 5)):
+        pairs = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(layers)]
+        step(k, pairs)
+        ev_all.append(pairs)
+    torch.cuda.synchronize()
+    call_times = [a.elapsed_time(b) / 1e3 for pairs in ev_all for a, b in pairs]
+    t_attn = float(np.mean(call_times))
+
+    elapsed_max = max_over_ranks(elapsed, world)
+    steps_total = sum_over_ranks(float(K), world)
+    value = steps_total / elapsed_max
+    accepted = float((lens_out[Wm:Wm + K].to(torch.int64) + 1).sum().item())
+    accepted_total = sum_over_ranks(accepted, world)
+    tok_s = accepted_total / elapsed_max
+
+    # accept-call timing
+    ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ea.record(stream)
+    for k in range(5):
+        acc.seed = k
+        acc.run(stream)
+    eb.record(stream)
+    torch.cuda.synchronize()
+    t_acc = ea.elapsed_time(eb) / 5e3
+
+    # roofline of the dominant call (attention)
+    kv_bytes = a0.kv_bytes_unique()
+    q_out = 2 * B * N * Hq * D * 2
+    tbl = int(sum((int(c) + 15) // 16 for c in a0.ctx_lens.tolist())) * 4
+    alg_bytes = kv_bytes + q_out + tbl
+    peak, peak_kind = measured_peaks()
+    achieved = alg_bytes / t_attn / 1e9
+    # accept: every logit once, plus one logit row and one draft row per sequence for the draw
+    acc_bytes = acc_in.target_logits.numel() * 4 + 8 * acc_in.vocab * B
+    step_bytes = layers * alg_bytes + acc_bytes
+
+    # e2e through the C-ABI with host buffers: inputs of a step copied H2D from
+    # pinned memory, results D2H, inside the timed region.
+    e2e = None
+    if not args.no_e2e:
+        host_q = [c.q.cpu().pin_memory() for c in calls]
+        host_l = acc_in.target_logits.pin_memory()
+        host_p = acc_in.draft_probs.pin_memory()
+        host_d = acc_in.draft_tokens.pin_memory()
+        host_t = a0.block_table.pin_memory()
+        host_c = a0.ctx_lens.pin_memory()
+        res_len = torch.empty((K, B), dtype=torch.int32).pin_memory()
+        res_tok = torch.empty((K, B), dtype=torch.int32).pin_memory()
+        h2d = (sum(h.numel() * h.element_size() for h in host_q) + host_l.numel() * 4 + host_p.numel() * 4
+               + host_d.numel() * 4 + host_t.numel() * 4 + host_c.numel() * 4)
+        d2h = 2 * B * 4
+
+        def e2e_step(k):
+            for c, h in zip(calls, host_q):
+                c.q.copy_(h, non_blocking=True)
+            calls[0].block_table.copy_(host_t, non_blocking=True)
+            calls[0].ctx_lens.copy_(host_c, non_blocking=True)
+            acc.logits.copy_(host_l, non_blocking=True)
+            acc.q.copy_(host_p, non_blocking=True)
+            acc.drafts.copy_(host_d, non_blocking=True)
+            for c in calls:
+                c.run(stream)
+            acc.seed = k
+            acc.accept_len = lens_out[k % (Wm + K)]
+            acc.run(stream)
+            res_len[k % K].copy_(acc.accept_len, non_blocking=True)
+            res_tok[k % K].copy_(acc.next_token, non_blocking=True)
+
+        for k in range(Wm):
+            e2e_step(k)
+        torch.cuda.synchronize()
+        barrier(world)
+        s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s2.record(stream)
+        for k in range(K):
+            e2e_step(k)
+        e2.record(stream)
+        torch.cuda.synchronize()
+        e2e_elapsed = max_over_ranks(s2.elapsed_time(e2) / 1e3, world)
+        e2e = {"value": steps_total / e2e_elapsed, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, ta, tc, sample = oracle_sample(w, a0, acc_in, layers, args.cpu_sample_seconds)
+        cpu = {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample,
+               "oracle_attn_layer_s": ta, "oracle_accept_s": tc}
+
+    clocks = clk.summary()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": Wm,
+            "ms_per_step": 1e3 * elapsed_max / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "layers": layers, "num_seqs": B, "gamma": N - 1,
+                       "q_heads": Hq, "kv_heads": a0.num_kv_heads, "head_dim": D,
+                       "ctx_tokens_total": int(a0.ctx_lens.sum()), "vocab": acc_in.vocab,
+                       "temperature": acc_in.temperature,
+                       "l2": "inputs larger than L2 (every layer has its own KV pool)",
+                       "parallelism": f"replicas x{world}"},
+            "accepted_tok_s": tok_s,
+            "t_attn_call_ms": 1e3 * t_attn, "t_accept_call_ms": 1e3 * t_acc,
+            "hbm_gbs_step": step_bytes / (elapsed_max / K) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                         "kernel": "sv_verify_attention (split + combine)",
+                         "algorithmic_bytes_per_call": alg_bytes, "peak_source": peak_kind},
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * (2 * layers + 1),
+            "clocks": clocks, "parity": parity,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        # host-only arm: rank 0 runs the oracle, other ranks exit without work
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
+    world, rank, local = dist_setup()
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

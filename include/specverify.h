@@ -1,0 +1,173 @@
+/*
+ * libspecverify -- the speculative-decoding verify step on one NVIDIA B200 (sm_100a).
+ *
+ * The verify step is the one target-model pass that scores all gamma+1 draft
+ * positions of every active rollout at once and then keeps the longest
+ * acceptable prefix (TLT reading notes, "1. RL and SD": the target scores
+ * d1..dgamma in one pass; once d1 fails, the results for later positions are
+ * discarded). Speculative decoding is used in RL rollouts because this step
+ * is lossless: it leaves the target's output distribution unchanged
+ * (Accelerating RL Post-Training Rollouts via System-Integrated Speculative
+ * Decoding, Abstract). The library implements the two parts of the step that
+ * touch every KV and logit byte:
+ *
+ *   sv_verify_attention  GQA attention of each sequence's N query rows (a
+ *                        causal chain of gamma+1 positions, or 1+nodes of a
+ *                        draft tree with per-row ancestor masks; SRT review,
+ *                        "Speculative Rollout integration", step 5) over a
+ *                        paged bf16 KV cache shared with the drafter
+ *                        (EfficientRollout, "Key modules" 1).
+ *   sv_accept            temperature softmax of the target logits, the accept
+ *                        test of each draft, the walk to the longest accepted
+ *                        path, and one token drawn from the residual
+ *                        norm(max(0, p - q)) (or from p when every draft on
+ *                        the path is accepted).
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, unless a
+ *     comment says host. Nothing is allocated, freed or retained by a call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Argument errors are detected on the host before any
+ *     launch and returned as sv_status; nothing is launched then.
+ *   - Data errors (bad context lengths, block ids, tokens, non-finite logits)
+ *     are reported per sequence in `status_flags` (SV_FLAG_* bits), written by
+ *     the kernels; read them after the stream is synchronised. Outputs of a
+ *     flagged sequence are defined below but carry no meaning.
+ *   - Calls that share a workspace must not overlap on the device.
+ *   - The library never reads or writes memory outside the ranges described
+ *     here; out-of-range block ids are never dereferenced.
+ */
+#ifndef SPECVERIFY_H
+#define SPECVERIFY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SV_API __attribute__((visibility("default")))
+#else
+#define SV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SV_OK = 0,
+    SV_ERR_INVALID_ARG = 1,   /* NULL/unaligned pointer, bad size or shape */
+    SV_ERR_UNSUPPORTED = 2,   /* valid request outside what the kernels handle */
+    SV_ERR_CUDA = 3,          /* a CUDA runtime call failed (see sv_last_error) */
+    SV_ERR_WORKSPACE = 4      /* workspace NULL or smaller than the size query */
+} sv_status;
+
+/* Per-sequence data-error bits written to status_flags[b]. */
+#define SV_FLAG_NONFINITE   1  /* accept: a NaN or +inf logit, or a row without a finite logit */
+#define SV_FLAG_BAD_CONTEXT 2  /* attention: ctx_len < N or ctx_len > max_blocks_per_seq*16 */
+#define SV_FLAG_BAD_TOKEN   4  /* accept: a draft token outside [0, vocab) */
+#define SV_FLAG_BAD_BLOCK   8  /* attention: a block id outside [0, num_blocks) */
+
+/* ------------------------------------------------------------------------
+ * Verify attention
+ * ------------------------------------------------------------------------
+ * Shapes (all row-major, contiguous):
+ *   q            bf16  [B][N][Hq][D]       query rows, RoPE already applied
+ *   k_pool/v_pool bf16 [num_blocks][Hkv][16][D]   paged KV pool (pages of 16 tokens)
+ *   block_table  int32 [B][max_blocks_per_seq]    page ids of each sequence
+ *   ctx_lens     int32 [B]                 keys of sequence b, INCLUDING its N new rows,
+ *                                          whose K/V the caller has already written
+ *   draft_mask   uint64 [B][N] or NULL     bit j of draft_mask[b][i]: row i sees new key j
+ *                                          (new key j = position ctx_len-N+j); NULL = chain
+ *                                          (row i sees new keys 0..i)
+ *   out          bf16  [B][N][Hq][D]
+ *   status_flags int32 [B] or NULL
+ * Query head hq reads KV head hq / (Hq/Hkv). Every row sees all prefix keys
+ * t < ctx_len - N. Scores are q.k / sqrt(D); out = softmax(scores) . V,
+ * accumulated in fp32. Limits: 1 <= N <= 64, D in {64, 128}, block_size 16,
+ * Hq % Hkv == 0, B <= 4096. q, out and the pools must be 16-byte aligned.
+ * A sequence flagged SV_FLAG_BAD_CONTEXT gets out = 0; one flagged
+ * SV_FLAG_BAD_BLOCK reads zeros for the bad pages. A row that sees no key
+ * gets out = 0.
+ * The work is split over the context across all SMs and then combined in a
+ * second kernel; `workspace` holds the per-split partials.
+ */
+typedef struct {
+    int32_t num_seqs;            /* B */
+    int32_t num_q_rows;          /* N = gamma+1 (chain) or 1+nodes (tree) */
+    int32_t num_q_heads;         /* Hq */
+    int32_t num_kv_heads;        /* Hkv */
+    int32_t head_dim;            /* D */
+    int32_t block_size;          /* tokens per page; must be 16 */
+    int32_t max_blocks_per_seq;  /* columns of block_table */
+    int32_t num_blocks;          /* pages in each pool */
+} sv_attn_desc;
+
+typedef struct {
+    const void *k_pool;          /* bf16 [num_blocks][Hkv][16][D] */
+    const void *v_pool;          /* bf16 [num_blocks][Hkv][16][D] */
+} sv_paged_kv;
+
+/* Bytes of device workspace sv_verify_attention needs for `desc` on the
+ * current device; 0 on an invalid desc. */
+SV_API size_t sv_verify_attention_workspace_size(const sv_attn_desc *desc);
+
+SV_API sv_status sv_verify_attention(const sv_attn_desc *desc, const void *q, const sv_paged_kv *paged_kv,
+                              const int32_t *block_table, const int32_t *ctx_lens,
+                              const uint64_t *draft_mask, void *out, void *workspace,
+                              size_t workspace_bytes, int32_t *status_flags, void *stream);
+
+/* ------------------------------------------------------------------------
+ * Accept / resample
+ * ------------------------------------------------------------------------
+ * Shapes:
+ *   target_logits fp32 [B][N][V]   row v: target logits of the token after node v
+ *                                  (row 0: after the last accepted token)
+ *   draft_probs   fp32 [B][N-1][V] row c-1: distribution draft token c was drawn from
+ *   draft_tokens  int32 [B][N-1]   token of draft node c at column c-1
+ *   accept_len    int32 [B]        out: number of accepted drafts (depth of the final node)
+ *   next_token    int32 [B]        out: the token emitted after the accepted path
+ *   accept_path   int32 [B][N-1] or NULL   out: accepted node ids, then -1
+ *   status_flags  int32 [B] or NULL        out: SV_FLAG_* bits
+ * tree_parents is a HOST array of N entries (tree_parents[0] = -1,
+ * 0 <= tree_parents[c] < c), copied at the call; NULL = chain (parent c-1).
+ *
+ * Rule (temperature T > 0): p_v = softmax(l_v / T). The walk starts at the
+ * root with residual r = p_0. Children c of the current node v are tried in
+ * index order with u = U(seed; b, c, 0): accept iff u * q_c(d_c) < r(d_c)
+ * (i.e. u < min(1, r/q)); accepting moves to c with r = p_c; rejecting sets
+ * r = norm(max(0, r - q_c)) (p_v if that has no mass) and tries the next
+ * child. When no child is accepted, next_token = InvCDF(r, U(seed; b, v, 1)).
+ * For a chain this is: accept drafts while u_i < min(1, p_i/q_i), then draw
+ * from norm(max(0, p - q)) at the first rejection, or from p after the last
+ * draft. T == 0 (greedy): move to the first child whose token is argmax l_v
+ * (lowest index on ties); next_token = argmax at the final node; draft_probs
+ * is not read and may be NULL.
+ * U(seed; b, c, tag) = (w0 >> 8) * 2^-24 where w0 is word 0 of
+ * Philox4x32-10 with key {seed_lo32, seed_hi32} and counter {b, c, tag, 0}
+ * (Salmon et al., SC'11). InvCDF(w, u) is the smallest x with
+ * sum_{y<=x} w(y) > u * sum(w), else the last x with w(x) > 0.
+ * Arithmetic is fp32. A sequence flagged SV_FLAG_NONFINITE gets
+ * accept_len 0, next_token 0; a bad draft token counts as rejected.
+ * Limits: 1 <= N <= 64, 1 <= V <= 8*57344, B <= 2^31-1 with grid limits.
+ */
+typedef struct {
+    int32_t num_seqs;             /* B */
+    int32_t num_rows;             /* N = drafts + 1 */
+    int32_t vocab;                /* V */
+    const int32_t *tree_parents;  /* HOST [N] or NULL (chain) */
+} sv_accept_desc;
+
+SV_API sv_status sv_accept(const sv_accept_desc *desc, const float *target_logits, const float *draft_probs,
+                    const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
+                    int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
+                    int32_t *status_flags, void *stream);
+
+/* Diagnostics. */
+SV_API const char *sv_status_string(sv_status s);
+SV_API const char *sv_last_error(void);   /* detail of the calling thread's last non-OK return */
+SV_API int32_t sv_version(void);          /* major*10000 + minor*100 + patch */
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SPECVERIFY_H */

@@ -1,0 +1,161 @@
+"""Python binding of libspecverify (the speculative-decoding verify step on B200).
+
+Argument marshalling only: every step of the verify path runs in the CUDA
+kernels of ``libspecverify.so``. The functions keep the C names and argument
+order of ``include/specverify.h``; tensor arguments may be torch CUDA tensors
+(their ``data_ptr()`` is passed) or raw integer device addresses. There is no
+CPU fallback: the first call raises ImportError if the shared library is
+missing (the library is loaded lazily so that the input generator module can
+be imported on machines without it).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from typing import Optional, Sequence
+
+__all__ = [
+    "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc",
+    "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_accept",
+    "sv_status_string", "sv_last_error", "sv_version", "library_path",
+    "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SO = os.path.join(_HERE, "libspecverify.so")
+
+SV_OK, SV_ERR_INVALID_ARG, SV_ERR_UNSUPPORTED, SV_ERR_CUDA, SV_ERR_WORKSPACE = range(5)
+SV_FLAG_NONFINITE = 1
+SV_FLAG_BAD_CONTEXT = 2
+SV_FLAG_BAD_TOKEN = 4
+SV_FLAG_BAD_BLOCK = 8
+
+
+class SvError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{sv_status_string(status)}: {detail}")
+        self.status = status
+
+
+class SvAttnDesc(C.Structure):
+    _fields_ = [("num_seqs", C.c_int32), ("num_q_rows", C.c_int32), ("num_q_heads", C.c_int32),
+                ("num_kv_heads", C.c_int32), ("head_dim", C.c_int32), ("block_size", C.c_int32),
+                ("max_blocks_per_seq", C.c_int32), ("num_blocks", C.c_int32)]
+
+
+class SvPagedKV(C.Structure):
+    _fields_ = [("k_pool", C.c_void_p), ("v_pool", C.c_void_p)]
+
+
+class SvAcceptDesc(C.Structure):
+    _fields_ = [("num_seqs", C.c_int32), ("num_rows", C.c_int32), ("vocab", C.c_int32),
+                ("tree_parents", C.POINTER(C.c_int32))]
+
+
+def _load() -> C.CDLL:
+    if not os.path.exists(_SO):
+        raise ImportError(
+            f"libspecverify.so not found at {_SO}; build it with "
+            "`python -m speculative_decoding_rl_b200.build` (nvcc, sm_100a)")
+    L = C.CDLL(_SO)
+    P, i32, u64, f32, sz = C.c_void_p, C.c_int32, C.c_uint64, C.c_float, C.c_size_t
+    L.sv_verify_attention_workspace_size.argtypes = [C.POINTER(SvAttnDesc)]
+    L.sv_verify_attention_workspace_size.restype = sz
+    L.sv_verify_attention.argtypes = [C.POINTER(SvAttnDesc), P, C.POINTER(SvPagedKV), P, P, P, P, P, sz, P, P]
+    L.sv_verify_attention.restype = C.c_int
+    L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P]
+    L.sv_accept.restype = C.c_int
+    L.sv_status_string.argtypes = [C.c_int]
+    L.sv_status_string.restype = C.c_char_p
+    L.sv_last_error.argtypes = []
+    L.sv_last_error.restype = C.c_char_p
+    L.sv_version.argtypes = []
+    L.sv_version.restype = i32
+    return L
+
+
+_lib_handle = None
+
+
+def _L() -> C.CDLL:
+    global _lib_handle
+    if _lib_handle is None:
+        _lib_handle = _load()
+    return _lib_handle
+
+
+def library_path() -> str:
+    return _SO
+
+
+def _ptr(x) -> Optional[int]:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if hasattr(x, "data_ptr"):
+        if x.device.type != "cuda":
+            raise ValueError("tensor arguments must live on a CUDA device")
+        return x.data_ptr()
+    raise TypeError(f"expected a CUDA tensor or an int address, got {type(x)}")
+
+
+def _stream(s) -> Optional[int]:
+    if s is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    if isinstance(s, int):
+        return s
+    return s.cuda_stream
+
+
+def _check(st: int) -> None:
+    if st != SV_OK:
+        raise SvError(st, sv_last_error())
+
+
+def sv_status_string(status: int) -> str:
+    return _L().sv_status_string(int(status)).decode()
+
+
+def sv_last_error() -> str:
+    return _L().sv_last_error().decode()
+
+
+def sv_version() -> int:
+    return int(_L().sv_version())
+
+
+def sv_verify_attention_workspace_size(desc: SvAttnDesc) -> int:
+    return int(_L().sv_verify_attention_workspace_size(C.byref(desc)))
+
+
+def sv_verify_attention(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_table, ctx_lens, draft_mask,
+                        out, workspace, workspace_bytes: int, status_flags=None, stream=None) -> None:
+    _check(_L().sv_verify_attention(C.byref(desc), _ptr(q), C.byref(paged_kv), _ptr(block_table),
+                                    _ptr(ctx_lens), _ptr(draft_mask), _ptr(out), _ptr(workspace),
+                                    int(workspace_bytes), _ptr(status_flags), _stream(stream)))
+
+
+def sv_accept(desc: SvAcceptDesc, target_logits, draft_probs, draft_tokens, temperature: float,
+              philox_seed: int, accept_len, next_token, accept_path=None, status_flags=None,
+              stream=None) -> None:
+    _check(_L().sv_accept(C.byref(desc), _ptr(target_logits), _ptr(draft_probs), _ptr(draft_tokens),
+                          float(temperature), int(philox_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(accept_len),
+                          _ptr(next_token), _ptr(accept_path), _ptr(status_flags), _stream(stream)))
+
+
+def make_accept_desc(num_seqs: int, num_rows: int, vocab: int,
+                     tree_parents: Optional[Sequence[int]] = None) -> SvAcceptDesc:
+    """Build an SvAcceptDesc; the parents array is kept alive on the returned object."""
+    d = SvAcceptDesc(num_seqs, num_rows, vocab, None)
+    if tree_parents is not None:
+        arr = (C.c_int32 * len(tree_parents))(*[int(x) for x in tree_parents])
+        d.tree_parents = C.cast(arr, C.POINTER(C.c_int32))
+        d._parents_keepalive = arr
+    return d

@@ -1,0 +1,168 @@
+// C-ABI entry points of libspecverify: argument validation on the host, then
+// asynchronous launches on the caller's stream. See include/specverify.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "sv_internal.h"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+sv_status fail(sv_status s, const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+sv_status check_attn_desc(const sv_attn_desc *d) {
+    if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
+    if (d->num_seqs < 0) return fail(SV_ERR_INVALID_ARG, "num_seqs < 0");
+    if (d->num_q_rows < 1 || d->num_q_rows > 64) return fail(SV_ERR_INVALID_ARG, "num_q_rows must be in [1, 64]");
+    if (d->num_q_heads < 1 || d->num_kv_heads < 1 || d->num_q_heads % d->num_kv_heads)
+        return fail(SV_ERR_INVALID_ARG, "num_q_heads must be a positive multiple of num_kv_heads");
+    if (d->head_dim != 64 && d->head_dim != 128) return fail(SV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+    if (d->block_size != sv::PAGE) return fail(SV_ERR_UNSUPPORTED, "block_size must be 16");
+    if (d->max_blocks_per_seq < 1) return fail(SV_ERR_INVALID_ARG, "max_blocks_per_seq < 1");
+    if (d->num_blocks < 1) return fail(SV_ERR_INVALID_ARG, "num_blocks < 1");
+    if (d->num_seqs > sv::MAX_SEQS) return fail(SV_ERR_UNSUPPORTED, "num_seqs > 4096");
+    if ((long long)d->max_blocks_per_seq * sv::PAGE > (1LL << 30)) return fail(SV_ERR_UNSUPPORTED, "context too long");
+    const long long rows = (long long)d->num_q_rows * (d->num_q_heads / d->num_kv_heads);
+    const long long units = (long long)d->num_seqs * d->num_kv_heads * ((rows + sv::ROWS_MAX - 1) / sv::ROWS_MAX);
+    if (units > 65535) return fail(SV_ERR_UNSUPPORTED, "num_seqs * num_kv_heads * row chunks above 65535");
+    return SV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *sv_status_string(sv_status s) {
+    switch (s) {
+        case SV_OK: return "SV_OK";
+        case SV_ERR_INVALID_ARG: return "SV_ERR_INVALID_ARG";
+        case SV_ERR_UNSUPPORTED: return "SV_ERR_UNSUPPORTED";
+        case SV_ERR_CUDA: return "SV_ERR_CUDA";
+        case SV_ERR_WORKSPACE: return "SV_ERR_WORKSPACE";
+    }
+    return "SV_ERR_UNKNOWN";
+}
+
+const char *sv_last_error(void) { return g_last_error; }
+
+int32_t sv_version(void) { return 100; }
+
+size_t sv_verify_attention_workspace_size(const sv_attn_desc *d) {
+    if (check_attn_desc(d) != SV_OK) return 0;
+    const int ctas = sv::attention_num_ctas();
+    if (ctas <= 0) return 0;
+    return sv::attention_workspace_bytes(d->num_seqs, d->num_q_rows, d->num_q_heads, d->num_kv_heads,
+                                         d->head_dim, ctas);
+}
+
+sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_paged_kv *kv,
+                              const int32_t *block_table, const int32_t *ctx_lens,
+                              const uint64_t *draft_mask, void *out, void *workspace,
+                              size_t workspace_bytes, int32_t *status_flags, void *stream) {
+    sv_status s = check_attn_desc(d);
+    if (s != SV_OK) return s;
+    if (d->num_seqs == 0) return SV_OK;
+    if (!q || !kv || !kv->k_pool || !kv->v_pool || !block_table || !ctx_lens || !out)
+        return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(kv->k_pool, 16) || !aligned(kv->v_pool, 16))
+        return fail(SV_ERR_INVALID_ARG, "q, out and the KV pools must be 16-byte aligned");
+    if (!aligned(block_table, 4) || !aligned(ctx_lens, 4) || (status_flags && !aligned(status_flags, 4)) ||
+        (draft_mask && !aligned(draft_mask, 8)))
+        return fail(SV_ERR_INVALID_ARG, "misaligned table, length, mask or status pointer");
+    const int ctas = sv::attention_num_ctas();
+    if (ctas <= 0) return fail(SV_ERR_CUDA, "cannot query the current device");
+    const size_t need = sv::attention_workspace_bytes(d->num_seqs, d->num_q_rows, d->num_q_heads,
+                                                      d->num_kv_heads, d->head_dim, ctas);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);
+
+    sv::AttnParams p = {};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k_pool = static_cast<const uint16_t *>(kv->k_pool);
+    p.v_pool = static_cast<const uint16_t *>(kv->v_pool);
+    p.block_table = block_table;
+    p.ctx_lens = ctx_lens;
+    p.mask = draft_mask;
+    p.out = static_cast<uint16_t *>(out);
+    p.status = status_flags;
+    p.B = d->num_seqs;
+    p.N = d->num_q_rows;
+    p.Hq = d->num_q_heads;
+    p.Hkv = d->num_kv_heads;
+    p.D = d->head_dim;
+    p.G = p.Hq / p.Hkv;
+    p.R = p.N * p.G;
+    p.RC = (p.R + sv::ROWS_MAX - 1) / sv::ROWS_MAX;
+    p.rows_unit = p.R < sv::ROWS_MAX ? p.R : sv::ROWS_MAX;
+    p.max_blocks = d->max_blocks_per_seq;
+    p.num_blocks = d->num_blocks;
+    p.units = p.B * p.Hkv * p.RC;
+    p.num_ctas = ctas;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
+    const size_t plan = (((size_t)(p.B + 3) * 4) + 255) & ~(size_t)255;
+    p.ws_plan = static_cast<int32_t *>(workspace);
+    p.ws_partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + plan);
+    cudaError_t e = sv::launch_attention(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SV_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+    return SV_OK;
+}
+
+sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const float *draft_probs,
+                    const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
+                    int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
+                    int32_t *status_flags, void *stream) {
+    if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
+    if (d->num_seqs < 0) return fail(SV_ERR_INVALID_ARG, "num_seqs < 0");
+    if (d->num_rows < 1 || d->num_rows > 64) return fail(SV_ERR_INVALID_ARG, "num_rows must be in [1, 64]");
+    if (d->vocab < 1) return fail(SV_ERR_INVALID_ARG, "vocab < 1");
+    if (d->vocab > sv::accept_max_vocab()) return fail(SV_ERR_UNSUPPORTED, "vocab above %d", sv::accept_max_vocab());
+    if (d->num_seqs > 65535) return fail(SV_ERR_UNSUPPORTED, "num_seqs above 65535");
+    if (!(temperature >= 0.f) || isinf(temperature)) return fail(SV_ERR_INVALID_ARG, "temperature must be finite and >= 0");
+    const bool greedy = temperature == 0.f;
+    sv::AcceptParams p = {};
+    p.parent[0] = -1;
+    for (int c = 1; c < d->num_rows; ++c) {
+        const int par = d->tree_parents ? d->tree_parents[c] : c - 1;
+        if (par < 0 || par >= c) return fail(SV_ERR_INVALID_ARG, "tree_parents[%d] = %d is not in [0, %d)", c, par, c);
+        p.parent[c] = (int8_t)par;
+    }
+    if (d->tree_parents && d->tree_parents[0] != -1) return fail(SV_ERR_INVALID_ARG, "tree_parents[0] must be -1");
+    if (d->num_seqs == 0) return SV_OK;
+    if (!target_logits || !accept_len || !next_token) return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (d->num_rows > 1 && !draft_tokens) return fail(SV_ERR_INVALID_ARG, "draft_tokens is NULL");
+    if (d->num_rows > 1 && !greedy && !draft_probs) return fail(SV_ERR_INVALID_ARG, "draft_probs is NULL");
+    if (!aligned(target_logits, 4) || (draft_probs && !aligned(draft_probs, 4)) ||
+        (draft_tokens && !aligned(draft_tokens, 4)) || !aligned(accept_len, 4) || !aligned(next_token, 4) ||
+        (accept_path && !aligned(accept_path, 4)) || (status_flags && !aligned(status_flags, 4)))
+        return fail(SV_ERR_INVALID_ARG, "misaligned pointer");
+    p.logits = target_logits;
+    p.q = draft_probs;
+    p.drafts = draft_tokens;
+    p.accept_len = accept_len;
+    p.next_token = next_token;
+    p.accept_path = accept_path;
+    p.status = status_flags;
+    p.B = d->num_seqs;
+    p.N = d->num_rows;
+    p.V = d->vocab;
+    p.greedy = greedy ? 1 : 0;
+    p.log2e_over_T = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
+    p.key.k0 = (uint32_t)(philox_seed & 0xFFFFFFFFull);
+    p.key.k1 = (uint32_t)(philox_seed >> 32);
+    cudaError_t e = sv::launch_accept(p, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SV_ERR_CUDA, "accept launch: %s", cudaGetErrorString(e));
+    return SV_OK;
+}
+
+}  // extern "C"

@@ -1,4 +1,5 @@
 import os
+import shutil
 import sys
 
 import pytest
@@ -10,7 +11,14 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    config.addinivalue_line("markers", "slow: long-running CPU statistics")
+    # Build the oracle (gcc) and the CUDA library (nvcc cross-compiles without a
+    # GPU); both builds are skipped when the shared objects are up to date.
+    import oracle
+    oracle.build()
+    if shutil.which(os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")) or \
+            os.path.exists("/usr/local/cuda/bin/nvcc"):
+        from speculative_decoding_rl_b200 import build
+        build.build()
 
 
 def cuda_available() -> bool:

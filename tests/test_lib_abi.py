@@ -1,0 +1,120 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before any launch (no GPU needed)."""
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+import speculative_decoding_rl_b200 as sv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "specverify.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SV_API\s+[\w\s\*]*?\b(sv_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("sv_verify_attention", "sv_verify_attention_workspace_size", "sv_accept",
+              "sv_status_string", "sv_last_error", "sv_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.CDLL(sv.library_path())
+    out = subprocess.check_output(["nm", "-D", "--defined-only", sv.library_path()], text=True)
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+        assert n in exported, n
+
+
+def test_library_targets_sm100a_only():
+    out = subprocess.check_output(["/usr/local/cuda/bin/cuobjdump", "--list-elf", sv.library_path()],
+                                  text=True)
+    archs = set(re.findall(r"sm_\w+", out))
+    assert archs == {"sm_100a"}, archs
+
+
+def test_status_strings_and_version():
+    assert sv.sv_status_string(0) == "SV_OK"
+    assert sv.sv_status_string(4) == "SV_ERR_WORKSPACE"
+    assert sv.sv_version() >= 100
+
+
+def _attn_desc(**kw):
+    d = dict(num_seqs=2, num_q_rows=5, num_q_heads=8, num_kv_heads=2, head_dim=128, block_size=16,
+             max_blocks_per_seq=8, num_blocks=32)
+    d.update(kw)
+    return sv.SvAttnDesc(**d)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_rows=0), sv.SV_ERR_INVALID_ARG),
+    (dict(num_q_rows=65), sv.SV_ERR_INVALID_ARG),
+    (dict(num_q_heads=6, num_kv_heads=4), sv.SV_ERR_INVALID_ARG),
+    (dict(head_dim=96), sv.SV_ERR_UNSUPPORTED),
+    (dict(block_size=32), sv.SV_ERR_UNSUPPORTED),
+    (dict(num_seqs=-1), sv.SV_ERR_INVALID_ARG),
+    (dict(num_seqs=5000), sv.SV_ERR_UNSUPPORTED),
+    (dict(num_blocks=0), sv.SV_ERR_INVALID_ARG),
+])
+def test_attention_rejects_bad_descriptors(kw, status):
+    d = _attn_desc(**kw)
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_verify_attention(d, 16, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20)
+    assert e.value.status == status
+    assert sv.sv_verify_attention_workspace_size(d) == 0
+
+
+def test_attention_rejects_null_and_misaligned_pointers():
+    d = _attn_desc()
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_verify_attention(d, None, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_verify_attention(d, 8, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+
+
+def test_attention_with_no_sequences_is_a_no_op():
+    sv.sv_verify_attention(_attn_desc(num_seqs=0), None, sv.SvPagedKV(None, None), None, None, None,
+                           None, None, 0)
+
+
+@pytest.mark.parametrize("kw,parents,temp,status", [
+    (dict(num_rows=0), None, 1.0, sv.SV_ERR_INVALID_ARG),
+    (dict(num_rows=65), None, 1.0, sv.SV_ERR_INVALID_ARG),
+    (dict(vocab=0), None, 1.0, sv.SV_ERR_INVALID_ARG),
+    (dict(vocab=10_000_000), None, 1.0, sv.SV_ERR_UNSUPPORTED),
+    (dict(), [-1, 0, 2, 1], 1.0, sv.SV_ERR_INVALID_ARG),   # parent not before child
+    (dict(), [0, 0, 1, 2], 1.0, sv.SV_ERR_INVALID_ARG),    # root parent must be -1
+    (dict(), None, -1.0, sv.SV_ERR_INVALID_ARG),
+    (dict(), None, float("nan"), sv.SV_ERR_INVALID_ARG),
+    (dict(), None, float("inf"), sv.SV_ERR_INVALID_ARG),
+])
+def test_accept_rejects_bad_arguments(kw, parents, temp, status):
+    d = dict(num_seqs=2, num_rows=4, vocab=100)
+    d.update(kw)
+    desc = sv.make_accept_desc(d["num_seqs"], d["num_rows"], d["vocab"], parents)
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_accept(desc, 16, 16, 16, temp, 0, 16, 16, None, None, stream=0)
+    assert e.value.status == status
+
+
+def test_accept_requires_outputs_and_drafts():
+    desc = sv.make_accept_desc(2, 4, 100)
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_accept(desc, 16, 16, None, 1.0, 0, 16, 16, None, None, stream=0)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_accept(desc, 16, None, 16, 1.0, 0, 16, 16, None, None, stream=0)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_accept(desc, 16, 16, 16, 1.0, 0, None, 16, None, None, stream=0)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
