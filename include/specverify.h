@@ -162,6 +162,32 @@ SV_API sv_status sv_accept(const sv_accept_desc *desc, const float *target_logit
                     int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
                     int32_t *status_flags, void *stream);
 
+/* ------------------------------------------------------------------------
+ * Verify attention without a workspace argument
+ * ------------------------------------------------------------------------
+ * The source pages have no counterpart to this call; it exists for callers
+ * that cannot allocate device memory (an engine or framework that owns every
+ * device buffer and forbids allocation while it runs, a plugin handed only
+ * its inputs and outputs, a host thread that must not call cudaMalloc because
+ * it can synchronise the device). Same arguments and results as
+ * sv_verify_attention minus the workspace: the split-context partials go to a
+ * scratch array of SV_NOALLOC_SCRATCH_BYTES built into the library's device
+ * image (every GPU that loads the library holds it until the process exits).
+ * The call allocates nothing. A request whose workspace size
+ * (sv_verify_attention_workspace_size) exceeds the scratch is refused with
+ * SV_ERR_WORKSPACE before any launch.
+ * The first call on a device looks up that device's scratch address; make it
+ * before any stream capture. All calls on a device share the scratch, which
+ * keeps the last call's contents (nothing in it needs clearing); calls whose
+ * executions overlap on the GPU race on it and must be ordered by the caller.
+ */
+#define SV_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+SV_API sv_status sv_verify_attention_noalloc(const sv_attn_desc *desc, const void *q,
+                                             const sv_paged_kv *paged_kv, const int32_t *block_table,
+                                             const int32_t *ctx_lens, const uint64_t *draft_mask,
+                                             void *out, int32_t *status_flags, void *stream);
+
 /* Diagnostics. */
 SV_API const char *sv_status_string(sv_status s);
 SV_API const char *sv_last_error(void);   /* detail of the calling thread's last non-OK return */

@@ -16,7 +16,7 @@ from typing import Optional, Sequence
 
 __all__ = [
     "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc",
-    "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_accept",
+    "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
 ]
@@ -29,6 +29,7 @@ SV_FLAG_NONFINITE = 1
 SV_FLAG_BAD_CONTEXT = 2
 SV_FLAG_BAD_TOKEN = 4
 SV_FLAG_BAD_BLOCK = 8
+SV_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class SvError(RuntimeError):
@@ -63,6 +64,8 @@ def _load() -> C.CDLL:
     L.sv_verify_attention_workspace_size.restype = sz
     L.sv_verify_attention.argtypes = [C.POINTER(SvAttnDesc), P, C.POINTER(SvPagedKV), P, P, P, P, P, sz, P, P]
     L.sv_verify_attention.restype = C.c_int
+    L.sv_verify_attention_noalloc.argtypes = [C.POINTER(SvAttnDesc), P, C.POINTER(SvPagedKV), P, P, P, P, P, P]
+    L.sv_verify_attention_noalloc.restype = C.c_int
     L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P]
     L.sv_accept.restype = C.c_int
     L.sv_status_string.argtypes = [C.c_int]
@@ -140,6 +143,16 @@ def sv_verify_attention(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_table, c
     _check(_L().sv_verify_attention(C.byref(desc), _ptr(q), C.byref(paged_kv), _ptr(block_table),
                                     _ptr(ctx_lens), _ptr(draft_mask), _ptr(out), _ptr(workspace),
                                     int(workspace_bytes), _ptr(status_flags), _stream(stream)))
+
+
+def sv_verify_attention_noalloc(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_table, ctx_lens,
+                                draft_mask, out, status_flags=None, stream=None) -> None:
+    """sv_verify_attention without a workspace argument, for callers that cannot
+    allocate device memory: the partials go to the library's built-in scratch
+    array (SV_NOALLOC_SCRATCH_BYTES). Calls that overlap on the GPU race on it."""
+    _check(_L().sv_verify_attention_noalloc(C.byref(desc), _ptr(q), C.byref(paged_kv), _ptr(block_table),
+                                            _ptr(ctx_lens), _ptr(draft_mask), _ptr(out), _ptr(status_flags),
+                                            _stream(stream)))
 
 
 def sv_accept(desc: SvAcceptDesc, target_logits, draft_probs, draft_tokens, temperature: float,

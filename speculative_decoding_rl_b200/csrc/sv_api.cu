@@ -41,6 +41,10 @@ sv_status check_attn_desc(const sv_attn_desc *d) {
 
 }  // namespace
 
+namespace sv {
+void record_error(const char *msg) { snprintf(g_last_error, sizeof g_last_error, "%s", msg); }
+}  // namespace sv
+
 extern "C" {
 
 const char *sv_status_string(sv_status s) {

@@ -61,4 +61,7 @@ size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_c
 int attention_num_ctas();
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
 
+// Sets the text sv_last_error() returns on the calling thread.
+void record_error(const char *msg);
+
 }  // namespace sv
