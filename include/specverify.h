@@ -66,6 +66,7 @@ typedef enum {
 #define SV_FLAG_BAD_CONTEXT 2  /* attention: ctx_len < N or ctx_len > max_blocks_per_seq*16 */
 #define SV_FLAG_BAD_TOKEN   4  /* accept: a draft token outside [0, vocab) */
 #define SV_FLAG_BAD_BLOCK   8  /* attention: a block id outside [0, num_blocks) */
+#define SV_FLAG_TIMEOUT    16  /* attention: a bounded device-side wait gave up; outputs invalid */
 
 /* ------------------------------------------------------------------------
  * Verify attention
@@ -83,13 +84,16 @@ typedef enum {
  *   status_flags int32 [B] or NULL
  * Query head hq reads KV head hq / (Hq/Hkv). Every row sees all prefix keys
  * t < ctx_len - N. Scores are q.k / sqrt(D); out = softmax(scores) . V,
- * accumulated in fp32. Limits: 1 <= N <= 64, D in {64, 128}, block_size 16,
- * Hq % Hkv == 0, B <= 4096. q, out and the pools must be 16-byte aligned.
+ * accumulated in fp32 (P is rounded to bf16 for the P.V tensor-core product).
+ * Limits: 1 <= N <= 64, D in {64, 128}, block_size 16, Hq % Hkv == 0,
+ * Hq/Hkv <= 96, B <= 1024. q, out and the pools must be 16-byte aligned.
  * A sequence flagged SV_FLAG_BAD_CONTEXT gets out = 0; one flagged
  * SV_FLAG_BAD_BLOCK reads zeros for the bad pages. A row that sees no key
  * gets out = 0.
- * The work is split over the context across all SMs and then combined in a
- * second kernel; `workspace` holds the per-split partials.
+ * The work is split over the context across all SMs (tcgen05 tensor cores,
+ * TMA page loads) and then combined in a second kernel; `workspace` holds the
+ * per-split partials. Device-side waits are bounded: if one gives up, every
+ * sequence of the call gets SV_FLAG_TIMEOUT.
  */
 typedef struct {
     int32_t num_seqs;            /* B */

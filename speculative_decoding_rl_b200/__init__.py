@@ -29,6 +29,7 @@ SV_FLAG_NONFINITE = 1
 SV_FLAG_BAD_CONTEXT = 2
 SV_FLAG_BAD_TOKEN = 4
 SV_FLAG_BAD_BLOCK = 8
+SV_FLAG_TIMEOUT = 16
 SV_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 

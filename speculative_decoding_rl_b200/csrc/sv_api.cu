@@ -31,10 +31,13 @@ sv_status check_attn_desc(const sv_attn_desc *d) {
     if (d->block_size != sv::PAGE) return fail(SV_ERR_UNSUPPORTED, "block_size must be 16");
     if (d->max_blocks_per_seq < 1) return fail(SV_ERR_INVALID_ARG, "max_blocks_per_seq < 1");
     if (d->num_blocks < 1) return fail(SV_ERR_INVALID_ARG, "num_blocks < 1");
-    if (d->num_seqs > sv::MAX_SEQS) return fail(SV_ERR_UNSUPPORTED, "num_seqs > 4096");
+    if (d->num_seqs > sv::MAX_SEQS) return fail(SV_ERR_UNSUPPORTED, "num_seqs > 1024");
+    if (d->num_q_heads / d->num_kv_heads > sv::ROWS_MAX)
+        return fail(SV_ERR_UNSUPPORTED, "more than 96 query heads per KV head");
     if ((long long)d->max_blocks_per_seq * sv::PAGE > (1LL << 30)) return fail(SV_ERR_UNSUPPORTED, "context too long");
-    const long long rows = (long long)d->num_q_rows * (d->num_q_heads / d->num_kv_heads);
-    const long long units = (long long)d->num_seqs * d->num_kv_heads * ((rows + sv::ROWS_MAX - 1) / sv::ROWS_MAX);
+    int ru, rc, nc;
+    sv::row_chunks(d->num_q_rows, d->num_q_heads / d->num_kv_heads, &ru, &rc, &nc);
+    const long long units = (long long)d->num_seqs * d->num_kv_heads * rc;
     if (units > 65535) return fail(SV_ERR_UNSUPPORTED, "num_seqs * num_kv_heads * row chunks above 65535");
     return SV_OK;
 }
@@ -107,14 +110,14 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
     p.D = d->head_dim;
     p.G = p.Hq / p.Hkv;
     p.R = p.N * p.G;
-    p.RC = (p.R + sv::ROWS_MAX - 1) / sv::ROWS_MAX;
-    p.rows_unit = p.R < sv::ROWS_MAX ? p.R : sv::ROWS_MAX;
+    int nc = 0;
+    sv::row_chunks(p.N, p.G, &p.rows_unit, &p.RC, &nc);
     p.max_blocks = d->max_blocks_per_seq;
     p.num_blocks = d->num_blocks;
     p.units = p.B * p.Hkv * p.RC;
     p.num_ctas = ctas;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
-    const size_t plan = (((size_t)(p.B + 3) * 4) + 255) & ~(size_t)255;
+    const size_t plan = sv::attention_plan_bytes(p.B);
     p.ws_plan = static_cast<int32_t *>(workspace);
     p.ws_partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + plan);
     cudaError_t e = sv::launch_attention(p, static_cast<cudaStream_t>(stream));

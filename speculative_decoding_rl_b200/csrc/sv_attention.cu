@@ -8,19 +8,52 @@
 // target (EfficientRollout, "Key modules" 1).
 //
 // Work decomposition (one persistent CTA per SM):
-//   unit  = (sequence b, KV head h, row chunk rc): the N*G query rows of the G
-//           query heads that read KV head h, at most ROWS_MAX per chunk;
+//   unit  = (sequence b, KV head h, row chunk rc): the query rows (i, g) of the
+//           G query heads that read KV head h; a chunk holds whole query rows
+//           i, at most ROWS_MAX rows (i, g) in all;
 //   tile  = TILE_KEYS consecutive keys of one unit;
-//   All tiles of all units are laid end to end and cut into num_ctas equal
+//   all tiles of all units are laid end to end and cut into num_ctas equal
 //   ranges, so every SM streams the same number of KV bytes whatever the mix
-//   of context lengths. Where a CTA's range covers part of a unit it writes a
-//   partial (unnormalised O, running max m, running sum l) to workspace slot
-//   unit + cta, which is unique because consecutive units can share at most
-//   one CTA. The combine kernel merges a unit's partials by their log-sum-exp.
-#include "sv_device.cuh"
+//   of context lengths. A CTA writes one partial (unnormalised O, running max
+//   m, running sum l; log2 domain) per unit it touches to workspace slot
+//   unit + cta, unique because consecutive units share at most one CTA; the
+//   combine kernel merges a unit's partials by their log-sum-exp.
+//
+// Inside a CTA (warp-specialised, tcgen05 + TMA, sm_100a):
+//   warp 0       TMA producer: per tile, 8 pages x {K, V} x (D/64) boxes of
+//                16 keys x 64 dims into a 128B-swizzled stage, plus the unit's
+//                query rows (one 3-D box per 64 dims) when a unit starts;
+//   warp 1       TMEM allocator and MMA issuer: S^T = K Q^T (M = 128 keys,
+//                N = padded rows RP, K = D) and O^T = V^T P^T (M = 128 dims,
+//                N = RP, K = 128 keys), fp32 accumulators in TMEM, S and O
+//                double-buffered;
+//   warps 2-9    two warpgroups, each owning half of the RP row columns: each
+//                thread owns one TMEM lane (a key for S, a head dim for O).
+//                Per tile: load S, mask, column max over the 128 keys (warp
+//                max + shared memory), online-softmax update, P (bf16) into a
+//                swizzled shared tile for the PV MMA, then rescale-and-add the
+//                previous tile's O^T into register accumulators.
+// Putting keys on the MMA M dimension keeps the tensor-core work at
+// 2 * 128 * RP * D per tile however few rows N*G there are, instead of
+// padding the rows to 128.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <string.h>
+
+#include <atomic>
+#include <mutex>
+
 #include "sv_internal.h"
+#include "sv_tc.cuh"
 
 namespace sv {
+
+using namespace tc;
+
+constexpr int TC_THREADS = 320;
+constexpr int MATH_THREADS_PER_WG = 128;
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
 
 // ---------------------------------------------------------------------------
 // Schedule helpers (attention and combine kernels agree on these).
@@ -38,7 +71,6 @@ SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch) {
     const int s0 = min(tid * per, p.B), s1 = min(s0 + per, p.B);
     int local = 0;
     for (int b = s0; b < s1; ++b) local += seq_tiles(p, b);
-    // block exclusive scan of `local`
     const int lane = tid & 31, warp = tid >> 5;
     int incl = local;
 #pragma unroll
@@ -59,9 +91,9 @@ SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch) {
     __syncthreads();
 }
 
-// Tile t -> sequence b (largest b with ups*TP[b] <= t), by binary search.
+// Tile t -> sequence b (largest b with ups*TP[b] <= t).
 SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
-    int lo = 0, hi = B;  // invariant: ups*TP[lo] <= t < ups*TP[hi]
+    int lo = 0, hi = B;
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
         if (ups * TP[mid] <= t) lo = mid; else hi = mid;
@@ -69,154 +101,418 @@ SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
     return lo;
 }
 
-SV_DEV bool key_visible(const AttnParams &p, int b, int C, int i, int t) {
-    if (t >= C) return false;
-    const int j = t - (C - p.N);
-    if (j < 0) return true;
-    if (p.mask) return (p.mask[(size_t)b * p.N + i] >> j) & 1ull;
-    return j <= i;
+struct TileInfo {
+    int b, hr, j, Tb;
+};
+
+SV_DEV TileInfo decode_tile(const int *TP, int B, int ups, int t) {
+    TileInfo ti;
+    ti.b = tile_seq(TP, B, ups, t);
+    ti.Tb = TP[ti.b + 1] - TP[ti.b];
+    const int off = t - ups * TP[ti.b];
+    ti.hr = off / ti.Tb;
+    ti.j = off - ti.hr * ti.Tb;
+    return ti;
 }
 
 // ---------------------------------------------------------------------------
-// Split-context attention on the CUDA cores: one page (16 keys) at a time,
-// fp32 in shared memory. Straightforward and exact to fp32 rounding.
+// Shared-memory plan of the tcgen05 kernel (host and device agree).
 // ---------------------------------------------------------------------------
-constexpr int V1_THREADS = 256;
+constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle column of a tile
 
-__global__ void __launch_bounds__(V1_THREADS, 1) attn_split_kernel(const AttnParams p) {
-    extern __shared__ __align__(16) float sm[];
-    const int D = p.D, RU = p.rows_unit;
-    int *TP = reinterpret_cast<int *>(sm);
-    int *scratch = TP + ((p.B + 1 + 3) & ~3);
-    float *Qs = reinterpret_cast<float *>(scratch + 32);
-    float *Ks = Qs + RU * D;
-    float *Vs = Ks + PAGE * (D + 1);
-    float *Ps = Vs + PAGE * D;
-    float *Os = Ps + RU * PAGE;
-    float *mrow = Os + RU * D;
-    float *lrow = mrow + RU;
-    float *arow = lrow + RU;
+struct TcLayout {
+    uint32_t stage_bytes, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_red, off_ms, off_as, off_lred,
+        off_misc, total;
+};
 
-    const int tid = threadIdx.x, nt = blockDim.x;
-    tile_prefix(p, TP, scratch);
+__host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, int B) {
+    TcLayout L;
+    const int nDA = D / 64;
+    const int RPh = RP / 2;
+    L.stage_bytes = 2u * nDA * ATOM;
+    L.off_q = NST * L.stage_bytes;
+    L.q_bytes = (uint32_t)nDA * RP * 128u;
+    L.off_p = L.off_q + 2u * L.q_bytes;
+    L.p_bytes = (uint32_t)((RP + 63) / 64) * ATOM;
+    L.off_bar = L.off_p + NP * L.p_bytes;
+    const int nbar = 2 * NST + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ + 2 /*wg*/;
+    L.off_tp = L.off_bar + 8u * nbar;
+    L.off_red = (L.off_tp + 4u * (B + 1) + 15u) & ~15u;
+    L.off_ms = L.off_red + 4u * 2 * 2 * 4 * RPh;   // [par][wg][warp][RPh]
+    L.off_as = L.off_ms + 4u * 2 * RP;             // [par][RP]
+    L.off_lred = L.off_as + 4u * 2 * RP;           // [par][RP]
+    L.off_misc = L.off_lred + 4u * 2 * 4 * RPh;    // [wg][warp][RPh]
+    L.total = L.off_misc + 64u;
+    return L;
+}
+
+struct TcParams {
+    CUtensorMap tm_k;
+    CUtensorMap tm_v;
+    CUtensorMap tm_q;
+    AttnParams a;
+    int NST, NP, Nc;
+    uint32_t epoch;
+};
+
+// ---------------------------------------------------------------------------
+// The tcgen05 split-context kernel.
+// ---------------------------------------------------------------------------
+template <int D, int RP>
+__global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams P) {
+    constexpr int nDA = D / 64;
+    constexpr int RPh = RP / 2;
+    constexpr int RPa = (RP + 31) / 32 * 32;  // TMEM columns per S / O buffer
+    const AttnParams &p = P.a;
+    const int NST = P.NST, NP = P.NP;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const TcLayout L = tc_layout(D, RP, NST, NP, p.B);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(base + L.off_bar);
+    uint64_t *kv_full = bar, *kv_empty = bar + NST;
+    uint64_t *q_full = bar + 2 * NST, *q_empty = q_full + 2;
+    uint64_t *s_full = q_empty + 2, *s_empty = s_full + 2;
+    uint64_t *p_full = s_empty + 2, *p_empty = p_full + NP;
+    uint64_t *o_full = p_empty + NP, *o_empty = o_full + 2;
+    uint64_t *done_bar = o_empty + 2;
+    uint64_t *wg_bar = done_bar + 1;  // warpgroup-local barriers of the two math warpgroups
+    int *TP = reinterpret_cast<int *>(base + L.off_tp);
+    float *red = reinterpret_cast<float *>(base + L.off_red);
+    float *mS = reinterpret_cast<float *>(base + L.off_ms);
+    float *aS = reinterpret_cast<float *>(base + L.off_as);
+    float *lred = reinterpret_cast<float *>(base + L.off_lred);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
+    int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // 10 ints, used once
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (tid == 0) {
+        for (int s = 0; s < NST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
+            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 2 * MATH_THREADS_PER_WG);
+            mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 2 * MATH_THREADS_PER_WG);
+        }
+        for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], 2 * MATH_THREADS_PER_WG); mbar_init(&p_empty[i], 1); }
+        mbar_init(done_bar, 1);
+        mbar_init(&wg_bar[0], MATH_THREADS_PER_WG);
+        mbar_init(&wg_bar[1], MATH_THREADS_PER_WG);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&P.tm_k);
+        tma_prefetch_desc(&P.tm_v);
+        tma_prefetch_desc(&P.tm_q);
+    }
+    {  // zero both query buffers: rows past a unit's real rows stay zero
+        uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
+        for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += TC_THREADS) q4[e] = make_uint4(0, 0, 0, 0);
+    }
+    tile_prefix(p, TP, scratch);  // contains __syncthreads
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
     const int ups = p.Hkv * p.RC;
     const int total = ups * TP[p.B];
-    if (total == 0) {
-        if (blockIdx.x == 0 && tid == 0) { p.ws_plan[0] = 1; p.ws_plan[1] = 0; }
-        if (blockIdx.x == 0) for (int b = tid; b <= p.B; b += nt) p.ws_plan[2 + b] = TP[b];
-        return;
-    }
-    const int W = (total + p.num_ctas - 1) / p.num_ctas;
+    const int W = total > 0 ? (total + p.num_ctas - 1) / p.num_ctas : 1;
     if (blockIdx.x == 0) {
         if (tid == 0) { p.ws_plan[0] = W; p.ws_plan[1] = total; }
-        for (int b = tid; b <= p.B; b += nt) p.ws_plan[2 + b] = TP[b];
+        for (int b = tid; b <= p.B; b += TC_THREADS) p.ws_plan[2 + b] = TP[b];
     }
-    const int t_begin = blockIdx.x * W;
+    const int t_begin = min((int)blockIdx.x * W, total);
     const int t_end = min(t_begin + W, total);
-    const size_t slot_floats = (size_t)RU * D + 2 * RU;
+    const int ntiles = t_end - t_begin;
 
-    int cur_u = -1, b = 0, h = 0, rc = 0, rows = 0, C = 0;
-    for (int t = t_begin; t <= t_end; ++t) {
-        int nb = 0, nhr = 0, j = 0, u = -1;
-        if (t < t_end) {
-            nb = tile_seq(TP, p.B, ups, t);
-            const int Tb = TP[nb + 1] - TP[nb];
-            const int off = t - ups * TP[nb];
-            nhr = off / Tb;
-            j = off - nhr * Tb;
-            u = nb * ups + nhr;
-        }
-        if (u != cur_u) {
-            if (cur_u >= 0) {  // flush the finished segment
-                float *slot = p.ws_partial + (size_t)(cur_u + blockIdx.x) * slot_floats;
-                for (int e = tid; e < rows * D; e += nt) slot[e] = Os[e];
-                for (int r = tid; r < rows; r += nt) {
-                    slot[(size_t)RU * D + r] = mrow[r];
-                    slot[(size_t)RU * D + RU + r] = lrow[r];
+    if (warp == 0) {
+        // ------------------------- TMA producer ---------------------------
+        if (lane == 0) {
+            const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
+            int lu = -1, issued_tiles = 0;
+            for (int lt = 0; lt < ntiles; ++lt) {
+                const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
+                const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
+                if (lt == 0 || ti.j == 0) {
+                    ++lu;
+                    const int qb = lu & 1;
+                    if (!mbar_wait(&q_empty[qb], ((lu >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                    mbar_arrive_expect_tx(&q_full[qb], q_box_bytes * nDA);
+                    uint8_t *qdst = base + L.off_q + qb * L.q_bytes;
+                    for (int a = 0; a < nDA; ++a)
+                        tma_load_3d(qdst + a * RP * 128, &P.tm_q, &q_full[qb], a * 64, h * p.G,
+                                    ti.b * p.N + rc * P.Nc);
                 }
-            }
-            if (u < 0) break;
-            cur_u = u;
-            b = nb;
-            h = nhr / p.RC;
-            rc = nhr - h * p.RC;
-            rows = min(ROWS_MAX, p.R - rc * ROWS_MAX);
-            C = p.ctx_lens[b];
-            __syncthreads();
-            for (int e = tid; e < rows * D; e += nt) {
-                const int r = e / D, d = e - r * D;
-                const int ridx = rc * ROWS_MAX + r;
-                const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
-                Qs[e] = bf16_bits_to_float(p.q[(((size_t)b * p.N + i) * p.Hq + hq) * D + d]);
-                Os[e] = 0.f;
-            }
-            for (int r = tid; r < rows; r += nt) { mrow[r] = -INFINITY; lrow[r] = 0.f; }
-            __syncthreads();
-        }
-        // ---- tile j of the unit: up to 8 pages ----
-        const int k0 = j * TILE_KEYS;
-        for (int pg = k0 / PAGE; pg < (k0 + TILE_KEYS) / PAGE; ++pg) {
-            const int t0 = pg * PAGE;
-            if (t0 >= C) break;
-            const int blk = p.block_table[(size_t)b * p.max_blocks + pg];
-            const bool bad = blk < 0 || blk >= p.num_blocks;
-            for (int e = tid; e < PAGE * D; e += nt) {
-                const int n = e / D, d = e - n * D;
-                float kv = 0.f, vv = 0.f;
-                if (!bad && t0 + n < C) {
-                    const size_t off = (((size_t)blk * p.Hkv + h) * PAGE + n) * D + d;
-                    kv = bf16_bits_to_float(p.k_pool[off]);
-                    vv = bf16_bits_to_float(p.v_pool[off]);
-                }
-                Ks[n * (D + 1) + d] = kv;
-                Vs[n * D + d] = vv;
-            }
-            __syncthreads();
-            for (int e = tid; e < rows * PAGE; e += nt) {
-                const int r = e >> 4, n = e & 15;
-                const int ridx = rc * ROWS_MAX + r;
-                const int i = ridx / p.G;
-                float s = -INFINITY;
-                if (key_visible(p, b, C, i, t0 + n)) {
-                    float acc = 0.f;
-                    const float *qr = Qs + r * D;
-                    const float *kr = Ks + n * (D + 1);
-                    for (int d = 0; d < D; ++d) acc = fmaf(qr[d], kr[d], acc);
-                    s = acc * p.scale_log2;
-                }
-                Ps[e] = s;
-            }
-            __syncthreads();
-            for (int r = tid; r < rows; r += nt) {
-                float mx = mrow[r];
-                for (int n = 0; n < PAGE; ++n) mx = fmaxf(mx, Ps[r * PAGE + n]);
-                float alpha = 1.f;
-                if (mx == -INFINITY) {
-                    for (int n = 0; n < PAGE; ++n) Ps[r * PAGE + n] = 0.f;
-                } else {
-                    alpha = exp2f(mrow[r] - mx);  // 0 when mrow is -inf
-                    float sum = 0.f;
-                    for (int n = 0; n < PAGE; ++n) {
-                        const float e = exp2f(Ps[r * PAGE + n] - mx);
-                        Ps[r * PAGE + n] = e;
-                        sum += e;
+                const int s = lt % NST;
+                if (!mbar_wait(&kv_empty[s], ((lt / NST) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                mbar_arrive_expect_tx(&kv_full[s], L.stage_bytes);
+                uint8_t *vdst = base + s * L.stage_bytes;
+                uint8_t *kdst = vdst + nDA * ATOM;
+                const int C = __ldg(p.ctx_lens + ti.b);
+                for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
+                    const int page = ti.j * (TILE_KEYS / PAGE) + pg;
+                    int blk = p.num_blocks;  // out of range: the TMA unit fills zeros
+                    if (page * PAGE < C) {
+                        const int x = __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page);
+                        if (x >= 0 && x < p.num_blocks) blk = x;
                     }
-                    lrow[r] = lrow[r] * alpha + sum;
-                    mrow[r] = mx;
+                    for (int a = 0; a < nDA; ++a) {
+                        tma_load_4d(vdst + a * ATOM + pg * 2048, &P.tm_v, &kv_full[s], a * 64, 0, h, blk);
+                        tma_load_4d(kdst + a * ATOM + pg * 2048, &P.tm_k, &kv_full[s], a * 64, 0, h, blk);
+                    }
                 }
-                arow[r] = alpha;
+                issued_tiles = lt + 1;
             }
-            __syncthreads();
-            for (int e = tid; e < rows * D; e += nt) {
-                const int r = e / D, d = e - r * D;
-                float o = Os[e] * arow[r];
-                const float *pr = Ps + r * PAGE;
-#pragma unroll
-                for (int n = 0; n < PAGE; ++n) o = fmaf(pr[n], Vs[n * D + d], o);
-                Os[e] = o;
+            if (*abort_flag) {
+                // let this CTA's own copies land before it can exit: the last
+                // use of every stage and query buffer must have completed
+                for (int lt = max(0, issued_tiles - NST); lt < issued_tiles; ++lt)
+                    mbar_wait_time(&kv_full[lt % NST], (lt / NST) & 1, WAIT_LIMIT_NS);
+                for (int u = max(0, lu - 1); u <= lu; ++u)
+                    mbar_wait_time(&q_full[u & 1], (u >> 1) & 1, WAIT_LIMIT_NS);
             }
-            __syncthreads();
         }
+    } else if (warp == 1) {
+        // -------------------------- MMA issuer ----------------------------
+        if (lane == 0) {
+            constexpr uint32_t idq = idesc_bf16(128, RP, false, false);
+            constexpr uint32_t idp = idesc_bf16(128, RP, true, true);
+            int lu = -1, qb = 0;
+            bool ok = true;
+            auto issue_pv = [&](int jt) -> bool {
+                const int s = jt % NST, pb = jt % NP, ob = jt & 1;
+                if (!mbar_wait(&p_full[pb], (jt / NP) & 1, abort_flag, WAIT_LIMIT_NS)) return false;
+                if (!mbar_wait(&o_empty[ob], ((jt >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) return false;
+                tc_fence_after();
+                const uint32_t va = smem_u32(base + s * L.stage_bytes);
+                const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
+#pragma unroll
+                for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(va + kk * 2048, ATOM, 1024);
+                    const uint64_t bd = sw128_desc(pa + kk * 2048, ATOM, 1024);
+                    mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, kk > 0);
+                }
+                mma_commit(&o_full[ob]);
+                mma_commit(&p_empty[pb]);
+                mma_commit(&kv_empty[s]);
+                return true;
+            };
+            for (int lt = 0; lt < ntiles && ok; ++lt) {
+                const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
+                const int s = lt % NST, sb = lt & 1;
+                if (lt == 0 || ti.j == 0) {
+                    ++lu;
+                    qb = lu & 1;
+                    if (!mbar_wait(&q_full[qb], (lu >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
+                }
+                if (!mbar_wait(&kv_full[s], (lt / NST) & 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
+                if (!mbar_wait(&s_empty[sb], ((lt >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t ka = smem_u32(base + s * L.stage_bytes + nDA * ATOM);
+                const uint32_t qa = smem_u32(base + L.off_q + qb * L.q_bytes);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t ad = sw128_desc(ka + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sw128_desc(qa + (kk >> 2) * (RP * 128) + (kk & 3) * 32, 16, 1024);
+                    mma_bf16_ss(tmem + sb * RPa, ad, bd, idq, kk > 0);
+                }
+                mma_commit(&s_full[sb]);
+                if (lt == ntiles - 1 || ti.j == ti.Tb - 1) mma_commit(&q_empty[qb]);
+                if (lt > 0) ok = issue_pv(lt - 1);
+            }
+            if (ok && ntiles > 0) issue_pv(ntiles - 1);
+            mma_commit(done_bar);  // every MMA of this CTA has finished before TMEM is freed
+            mbar_wait_time(done_bar, 0, WAIT_LIMIT_NS);
+        }
+    } else {
+        // ---------------------- softmax / correction ----------------------
+        const int wg = (warp - 2) >> 2;   // column half
+        const int wiw = (warp - 2) & 3;   // warp within the warpgroup
+        const int wq = warp & 3;          // TMEM lane quadrant this warp may access
+        const int ell = wq * 32 + lane;   // key (S) / head dim (O) lane
+        const int col0 = wg * RPh;
+        uint32_t wg_phase = 0;
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        float acc[RPh], lsum[RPh];
+#pragma unroll
+        for (int c = 0; c < RPh; ++c) { acc[c] = 0.f; lsum[c] = 0.f; }
+        const size_t slot_floats = (size_t)p.rows_unit * D + 2 * p.rows_unit;
+        bool ok = true;
+
+        int cur_u = -1, last_par = 0;
+        int ub = 0, uh = 0, urc = 0, uC = 0, urows = 0;
+
+        // warp-uniform bounded wait: the tcgen05 loads that follow are .sync.aligned
+        auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
+            const bool r = mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
+            return __all_sync(0xffffffffu, r);
+        };
+        auto correction = [&](int jt) -> bool {
+            const int ob = jt & 1;
+            if (!wait_w(&o_full[ob], (jt >> 1) & 1)) return false;
+            tc_fence_after();
+            float o[RPh];
+            tmem_ld_cols<RPh>(lane_base + (2 + ob) * RPa + col0, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&o_empty[ob]);
+            const float *al = aS + (jt & 1) * RP + col0;
+#pragma unroll
+            for (int c = 0; c < RPh; ++c) acc[c] = fmaf(acc[c], al[c], o[c]);
+            return true;
+        };
+        auto wg_sync = [&]() -> bool {
+            mbar_arrive(&wg_bar[wg]);
+            const bool r = wait_w(&wg_bar[wg], wg_phase);
+            wg_phase ^= 1;
+            return r;
+        };
+        auto finalize = [&]() -> bool {
+#pragma unroll
+            for (int c = 0; c < RPh; ++c) {
+                const float v = warp_sum(lsum[c]);
+                if (lane == 0) lred[(wg * 4 + wiw) * RPh + c] = v;
+            }
+            if (!wg_sync()) return false;
+            float *slot = p.ws_partial + (size_t)(cur_u + blockIdx.x) * slot_floats;
+            if (ell < D) {
+#pragma unroll
+                for (int c = 0; c < RPh; ++c)
+                    if (col0 + c < urows) slot[(size_t)(col0 + c) * D + ell] = acc[c];
+            }
+            if (wiw == 0) {
+                for (int c = lane; c < RPh; c += 32) {
+                    const int r = col0 + c;
+                    if (r < urows) {
+                        float l = 0.f;
+                        for (int w = 0; w < 4; ++w) l += lred[(wg * 4 + w) * RPh + c];
+                        slot[(size_t)p.rows_unit * D + r] = mS[last_par * RP + r];
+                        slot[(size_t)p.rows_unit * D + p.rows_unit + r] = l;
+                    }
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < RPh; ++c) { acc[c] = 0.f; lsum[c] = 0.f; }
+            return true;
+        };
+
+        for (int lt = 0; lt < ntiles && ok; ++lt) {
+            const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
+            const bool first = (lt == 0 || ti.j == 0);
+            if (first) {
+                if (lt > 0) {
+                    if (!(ok = correction(lt - 1))) break;
+                    if (!(ok = finalize())) break;
+                }
+                cur_u = ti.b * ups + ti.hr;
+                ub = ti.b;
+                uh = ti.hr / p.RC;
+                urc = ti.hr - uh * p.RC;
+                uC = __ldg(p.ctx_lens + ub);
+                urows = min(p.rows_unit, p.R - urc * p.rows_unit);
+            }
+            // ---- softmax of tile lt ----
+            const int sb = lt & 1, par = lt & 1;
+            if (!(ok = wait_w(&s_full[sb], (lt >> 1) & 1))) break;
+            tc_fence_after();
+            float sv[RPh];
+            tmem_ld_cols<RPh>(lane_base + sb * RPa + col0, sv);
+            tmem_wait_ld();
+            tc_fence_before();
+            mbar_arrive(&s_empty[sb]);
+
+            const int key = ti.j * TILE_KEYS + ell;
+            const bool valid = key < uC;
+            const int newk = key - (uC - p.N);
+#pragma unroll
+            for (int c = 0; c < RPh; ++c) {
+                float v = sv[c] * p.scale_log2;
+                if (!valid) {
+                    v = -INFINITY;
+                } else if (newk >= 0 && col0 + c < urows) {
+                    const int i = urc * P.Nc + (col0 + c) / p.G;
+                    const bool vis = p.mask ? ((__ldg(p.mask + (size_t)ub * p.N + i) >> newk) & 1ull) != 0
+                                            : newk <= i;
+                    if (!vis) v = -INFINITY;
+                }
+                sv[c] = v;
+            }
+            float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
+#pragma unroll
+            for (int c = 0; c < RPh; ++c) {
+                const float m = warp_max(sv[c]);
+                if (lane == 0) rd[c] = m;
+            }
+            if (!(ok = wg_sync())) break;
+            if (wiw == 0) {
+                for (int c = lane; c < RPh; c += 32) {
+                    const float mo = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
+                    float mx = mo;
+                    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, red[((par * 2 + wg) * 4 + w) * RPh + c]);
+                    mS[par * RP + col0 + c] = mx;
+                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : exp2f(mo - mx);
+                }
+            }
+            if (!(ok = wg_sync())) break;
+            last_par = par;
+            const float *ms = mS + par * RP + col0;
+            const float *as = aS + par * RP + col0;
+            uint32_t packed[RPh / 2];
+#pragma unroll
+            for (int c = 0; c < RPh; c += 2) {
+                const float m0 = ms[c], m1 = ms[c + 1];
+                const float p0 = (m0 == -INFINITY) ? 0.f : exp2f(sv[c] - m0);
+                const float p1 = (m1 == -INFINITY) ? 0.f : exp2f(sv[c + 1] - m1);
+                lsum[c] = fmaf(lsum[c], as[c], p0);
+                lsum[c + 1] = fmaf(lsum[c + 1], as[c + 1], p1);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                packed[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
+            }
+            const int pb = lt % NP;
+            if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
+            uint8_t *pbuf = base + L.off_p + pb * L.p_bytes;
+#pragma unroll
+            for (int c8 = 0; c8 < RPh / 8; ++c8) {
+                const int cc = col0 + c8 * 8;
+                const int chunk = (cc & 63) >> 3;
+                uint4 *dst = reinterpret_cast<uint4 *>(pbuf + (cc >> 6) * ATOM + (ell >> 3) * 1024 +
+                                                       (ell & 7) * 128 + ((chunk ^ (ell & 7)) << 4));
+                *dst = make_uint4(packed[c8 * 4], packed[c8 * 4 + 1], packed[c8 * 4 + 2], packed[c8 * 4 + 3]);
+            }
+            if (!valid && wg == 0) {
+                // a key past ctx_len: its V row may hold anything (NaN) and P = 0 does not cancel it
+                uint8_t *vrow = base + (lt % NST) * L.stage_bytes + ell * 128;
+                for (int a = 0; a < nDA; ++a)
+                    for (int q = 0; q < 8; ++q)
+                        reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&p_full[pb]);
+            // ---- rescale-and-add the previous tile of the same unit ----
+            if (!first)
+                if (!(ok = correction(lt - 1))) break;
+        }
+        if (ok && ntiles > 0) {
+            if (correction(ntiles - 1)) finalize();
+        }
+    }
+
+    // ----------------------------- teardown -------------------------------
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && tid == 0) atomicExch(reinterpret_cast<unsigned int *>(p.ws_plan + p.B + 3), P.epoch);
+    if (warp == 1) {
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
     }
 }
 
@@ -225,15 +521,15 @@ __global__ void __launch_bounds__(V1_THREADS, 1) attn_split_kernel(const AttnPar
 // (row of a unit, unit), one thread per head dimension. The CTA of row 0 of
 // each sequence's first unit also writes that sequence's status flags.
 // ---------------------------------------------------------------------------
-__global__ void attn_combine_kernel(const AttnParams p) {
+__global__ void attn_combine_kernel(const AttnParams p, uint32_t epoch) {
     const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x;
     const int D = p.D, RU = p.rows_unit;
     const int ups = p.Hkv * p.RC;
     const int b = u / ups, hr = u - b * ups;
     const int h = hr / p.RC, rc = hr - h * p.RC;
-    const int rows = min(ROWS_MAX, p.R - rc * ROWS_MAX);
+    const int rows = min(RU, p.R - rc * RU);
     if (r >= rows) return;
-    const int ridx = rc * ROWS_MAX + r;
+    const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const int W = p.ws_plan[0];
     const int *TP = p.ws_plan + 2;
@@ -272,18 +568,31 @@ __global__ void attn_combine_kernel(const AttnParams p) {
                 bad |= (blk < 0 || blk >= p.num_blocks);
             }
         bad = __syncthreads_or(bad);
-        if (d == 0) p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0);
+        if (d == 0) {
+            const bool timed_out = (uint32_t)p.ws_plan[p.B + 3] == epoch;
+            p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0) |
+                          (timed_out ? SV_FLAG_TIMEOUT : 0);
+        }
     }
 }
 
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-static size_t plan_bytes(int B) { return (((size_t)(B + 3) * 4) + 255) & ~(size_t)255; }
+static size_t plan_bytes(int B) { return (((size_t)(B + 4) * 4) + 255) & ~(size_t)255; }
 
-static int rows_per_unit(int N, int Hq, int Hkv) {
-    const int R = N * (Hq / Hkv);
-    return R < ROWS_MAX ? R : ROWS_MAX;
+void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc) {
+    const int R = N * G;
+    if (R <= ROWS_MAX) {
+        *rows_unit = R;
+        *RC = 1;
+        *Nc = N;
+    } else {
+        const int nc = ROWS_MAX / G;  // whole query rows per chunk (G <= ROWS_MAX is validated)
+        *Nc = nc;
+        *rows_unit = nc * G;
+        *RC = (N + nc - 1) / nc;
+    }
 }
 
 int attention_num_ctas() {
@@ -294,27 +603,109 @@ int attention_num_ctas() {
 }
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas) {
-    const int R = N * (Hq / Hkv);
-    const int RC = (R + ROWS_MAX - 1) / ROWS_MAX;
-    const int RU = rows_per_unit(N, Hq, Hkv);
+    int RU, RC, Nc;
+    row_chunks(N, Hq / Hkv, &RU, &RC, &Nc);
     const size_t units = (size_t)B * Hkv * RC;
     const size_t slot_floats = (size_t)RU * D + 2 * RU;
     return plan_bytes(B) + (units + (size_t)num_ctas) * slot_floats * sizeof(float);
 }
 
-cudaError_t launch_attention(const AttnParams &p0, cudaStream_t stream) {
-    AttnParams p = p0;
-    const int D = p.D, RU = p.rows_unit;
-    const size_t smem = sizeof(int) * ((size_t)((p.B + 1 + 3) & ~3) + 32) +
-                        sizeof(float) * ((size_t)RU * D + PAGE * (D + 1) + PAGE * D + RU * PAGE +
-                                         (size_t)RU * D + 3 * RU);
-    cudaError_t e = cudaFuncSetAttribute(attn_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+size_t attention_plan_bytes(int B) { return plan_bytes(B); }
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+static bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)PAGE, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
+    const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)PAGE * D * 2, (cuuint64_t)Hkv * PAGE * D * 2};
+    const cuuint32_t box[4] = {64, PAGE, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pool), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static bool encode_q_map(CUtensorMap *m, const void *q, int B, int N, int Hq, int D, int G, int Nc) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)Hq, (cuuint64_t)B * N};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Hq * D * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)G, (cuuint32_t)Nc};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(q), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr int SMEM_LIMIT = 227 * 1024;
+
+template <int D, int RP>
+static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
+    // two KV stages at D=128 (four at D=64), double-buffered P when it fits
+    int NST = D == 128 ? 2 : 4;
+    int NP = 2;
+    TcLayout L = tc_layout(D, RP, NST, NP, P.a.B);
+    if (L.total + 1024 > (uint32_t)SMEM_LIMIT) {
+        NP = 1;
+        L = tc_layout(D, RP, NST, NP, P.a.B);
+    }
+    if (L.total + 1024 > (uint32_t)SMEM_LIMIT) return cudaErrorInvalidConfiguration;
+    P.NST = NST;
+    P.NP = NP;
+    const size_t smem = L.total + 1024;
+    auto kfn = attn_tc_kernel<D, RP>;
+    cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    attn_split_kernel<<<p.num_ctas, V1_THREADS, smem, stream>>>(p);
-    e = cudaGetLastError();
+    kfn<<<P.a.num_ctas, TC_THREADS, smem, stream>>>(P);
+    return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_tc_rp(TcParams &P, int RP, cudaStream_t stream) {
+    switch (RP) {
+        case 16: return launch_tc<D, 16>(P, stream);
+        case 32: return launch_tc<D, 32>(P, stream);
+        case 48: return launch_tc<D, 48>(P, stream);
+        case 64: return launch_tc<D, 64>(P, stream);
+        case 80: return launch_tc<D, 80>(P, stream);
+        case 96: return launch_tc<D, 96>(P, stream);
+    }
+    return cudaErrorInvalidValue;
+}
+
+static uint32_t next_epoch() {
+    static std::atomic<uint32_t> e{0x5A000000u};
+    return ++e;
+}
+
+cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
+    TcParams P;
+    memset(&P, 0, sizeof P);
+    P.a = p;
+    int RU, RC, Nc;
+    row_chunks(p.N, p.G, &RU, &RC, &Nc);
+    P.Nc = Nc;
+    P.epoch = next_epoch();
+    if (!encode_pool_map(&P.tm_k, p.k_pool, p.num_blocks, p.Hkv, p.D) ||
+        !encode_pool_map(&P.tm_v, p.v_pool, p.num_blocks, p.Hkv, p.D) ||
+        !encode_q_map(&P.tm_q, p.q, p.B, p.N, p.Hq, p.D, p.G, Nc))
+        return cudaErrorInvalidValue;
+    const int RP = (RU + 15) / 16 * 16;
+    cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3(RU, p.units), D, 0, stream>>>(p);
+    attn_combine_kernel<<<dim3(RU, p.units), p.D, 0, stream>>>(p, P.epoch);
     return cudaGetLastError();
 }
 

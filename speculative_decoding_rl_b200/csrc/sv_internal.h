@@ -37,8 +37,8 @@ cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream);
 // keys of one (sequence, KV head, row chunk) unit.
 constexpr int TILE_KEYS = 128;
 constexpr int PAGE = 16;
-constexpr int ROWS_MAX = 128;      // query rows (N*G) one unit carries
-constexpr int MAX_SEQS = 4096;
+constexpr int ROWS_MAX = 96;       // query rows (N*G) one unit carries
+constexpr int MAX_SEQS = 1024;
 
 struct AttnParams {
     const uint16_t *q;         // bf16 bits [B][N][Hq][D]
@@ -50,7 +50,8 @@ struct AttnParams {
     uint16_t *out;             // bf16 bits [B][N][Hq][D]
     int32_t *status;           // [B] or null
     float *ws_partial;         // slots x (rows*D + 2*rows) floats
-    int32_t *ws_plan;          // [0] = tiles per CTA, [1] = total tiles, [2..2+B] = tile prefix per sequence
+    int32_t *ws_plan;          // [0] tiles per CTA, [1] total tiles, [2..2+B] tile prefix per sequence,
+                               // [B+3] epoch of the last call that timed out
     int B, N, Hq, Hkv, D, G, R, RC, rows_unit, max_blocks, num_blocks;
     int units;                 // B * Hkv * RC
     int num_ctas;
@@ -58,6 +59,9 @@ struct AttnParams {
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
+size_t attention_plan_bytes(int B);
+// Row chunks of a unit: rows_unit rows (i, g) per chunk, RC chunks, Nc whole query rows i per chunk.
+void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc);
 int attention_num_ctas();
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
 
