@@ -49,7 +49,7 @@ def lib() -> C.CDLL:
         L.orc_attention.restype = i32
         L.orc_attention_rows.argtypes = [i32] * 8 + [P] * 6 + [P, i32, P]
         L.orc_attention_rows.restype = i32
-        L.orc_accept.argtypes = [i32, i32, i32, P, P, P, P, f64, u64, P, P, P, P, P, P]
+        L.orc_accept.argtypes = [i32, i32, i32, P, P, P, P, f64, u64, P, P, P, P, P, P, P, P]
         L.orc_accept.restype = i32
         L.orc_inv_cdf.argtypes = [P, i32, f64, P]
         L.orc_inv_cdf.restype = i32
@@ -130,6 +130,8 @@ class AcceptResult:
         self.next_token = np.zeros(B, dtype=np.int32)
         self.tie_depth = np.full(B, -1, dtype=np.int32)
         self.tie_draw = np.zeros(B, dtype=np.int32)
+        self.draw_lo = np.zeros(B, dtype=np.int32)
+        self.draw_hi = np.zeros(B, dtype=np.int32)
         self.flags = np.zeros(B, dtype=np.int32)
 
 
@@ -149,7 +151,8 @@ def accept(logits, draft_probs, draft_tokens, temperature: float, seed: int,
     path = res.accept_path if N > 1 else np.zeros((B, 1), dtype=np.int32)
     rc = lib().orc_accept(B, N, V, _p(par), _p(l), _p(q), _p(d), float(temperature), int(seed),
                           _p(res.accept_len), _p(path), _p(res.next_token),
-                          _p(res.tie_depth), _p(res.tie_draw), _p(res.flags))
+                          _p(res.tie_depth), _p(res.tie_draw), _p(res.draw_lo), _p(res.draw_hi),
+                          _p(res.flags))
     if rc:
         raise ValueError(f"orc_accept returned {rc}")
     return res

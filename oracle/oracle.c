@@ -245,6 +245,19 @@ static int row_argmax(const float *l, int V)
     return best;
 }
 
+/* Smallest x with sum_{y<=x} w(y) > t (t absolute), else the last x with w(x) > 0. */
+static int first_above(const double *w, int V, double t)
+{
+    double c = 0.0;
+    for (int x = 0; x < V; ++x) {
+        c += w[x];
+        if (c > t) return x;
+    }
+    for (int x = V - 1; x >= 0; --x)
+        if (w[x] > 0.0) return x;
+    return V - 1;
+}
+
 /* Inverse CDF over unnormalised weights w >= 0: the smallest x with
  * sum_{y<=x} w(y) > u * sum(w); if rounding leaves none, the last x with
  * w(x) > 0. *gap gets the distance from u*sum(w) to the nearer end of x's
@@ -295,14 +308,17 @@ static int inv_cdf(const double *w, int V, double u, double *gap)
  * [B][N-1] (the accepted nodes, -1 after the end), next_token, and for
  * parity accounting tie_depth (depth of the node at which the first accept
  * test with |u - r(d)/q(d)| < 1e-5 happened, else -1), tie_draw (1 if the
- * final draw's gap < 1e-5 and no accept test was a near tie) and flags
+ * final draw's gap < 1e-5 and no accept test was a near tie), draw_lo /
+ * draw_hi (the tokens the draw picks at thresholds (u -/+ 1e-5) * sum(w):
+ * every token a rounding of the threshold within that band can give) and flags
  * (bit 0: non-finite logits, bit 2: bad draft token).
  * Returns 0, or a negative value on bad arguments / allocation failure.
  */
 int orc_accept(int B, int N, int V, const int32_t *parents, const float *logits,
                const float *draft_probs, const int32_t *drafts, double T, uint64_t seed,
                int32_t *accept_len, int32_t *accept_path, int32_t *next_token,
-               int32_t *tie_depth, int32_t *tie_draw, int32_t *flags)
+               int32_t *tie_depth, int32_t *tie_draw, int32_t *draw_lo, int32_t *draw_hi,
+               int32_t *flags)
 {
     if (B < 0 || N < 1 || N > 64 || V < 1 || T < 0.0) return -2;
     int *par = (int *)malloc(sizeof(int) * (size_t)N);
@@ -320,7 +336,7 @@ int orc_accept(int B, int N, int V, const int32_t *parents, const float *logits,
         const int32_t *db = drafts + (size_t)b * (N - 1);
         int32_t *path = accept_path + (size_t)b * (N - 1);
         for (int k = 0; k < N - 1; ++k) path[k] = -1;
-        int v = 0, depth = 0, flag = 0, tdepth = -1, tdraw = 0, tok = 0;
+        int v = 0, depth = 0, flag = 0, tdepth = -1, tdraw = 0, tok = 0, dlo = 0, dhi = 0;
         for (int row = 0; row < N; ++row)
             if (row_argmax(lb + (size_t)row * V, V) < 0) flag |= 1;
         if (flag) goto done;
@@ -377,12 +393,18 @@ int orc_accept(int B, int N, int V, const int32_t *parents, const float *logits,
             double u = orc_uniform(seed, (uint32_t)b, (uint32_t)v, 1u, 0u);
             tok = inv_cdf(r, V, u, &gap);
             if (tdepth < 0 && gap < ORC_TIE_EPS) tdraw = 1;
+            double total = 0.0;
+            for (int x = 0; x < V; ++x) total += r[x];
+            dlo = first_above(r, V, (u - ORC_TIE_EPS) * total);
+            dhi = first_above(r, V, (u + ORC_TIE_EPS) * total);
         }
     done:
         accept_len[b] = depth;
         next_token[b] = tok;
         if (tie_depth) tie_depth[b] = tdepth;
         if (tie_draw) tie_draw[b] = tdraw;
+        if (draw_lo) draw_lo[b] = T == 0.0 ? tok : dlo;
+        if (draw_hi) draw_hi[b] = T == 0.0 ? tok : dhi;
         if (flags) flags[b] = flag;
     }
     free(par); free(r); free(pv);

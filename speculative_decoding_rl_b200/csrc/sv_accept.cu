@@ -283,12 +283,40 @@ __global__ void __launch_bounds__(ACC_THREADS, 1) accept_kernel(const AcceptPara
             if (dsib < lo || dsib >= hi) dsib = -1;
         }
         float part = 0.f;
-        for (int x = tid; x < n; x += ACC_THREADS) {
-            const float r = from_p ? exp2f((__ldg(lrow + lo + x) - Mv) * c) / Sv : rbuf[x] / rZ;
-            const float w = fmaxf(r - __ldg(qrow + lo + x), 0.f);
-            rbuf[x] = w;
-            part += w;
-            if (lo + x == dsib) S.slot[S.parity].rnext = w;
+        if (VEC) {
+            // n and lo are multiples of 4 and the rows are 16-byte aligned
+            const float4 *l4 = reinterpret_cast<const float4 *>(lrow + lo);
+            const float4 *q4 = reinterpret_cast<const float4 *>(qrow + lo);
+            float4 *r4 = reinterpret_cast<float4 *>(rbuf);
+#pragma unroll 4
+            for (int x = tid; x < (n >> 2); x += ACC_THREADS) {
+                const float4 qv = __ldg(q4 + x);
+                float4 rv;
+                if (from_p) {
+                    const float4 lv = __ldg(l4 + x);
+                    rv = make_float4(exp2f((lv.x - Mv) * c) / Sv, exp2f((lv.y - Mv) * c) / Sv,
+                                     exp2f((lv.z - Mv) * c) / Sv, exp2f((lv.w - Mv) * c) / Sv);
+                } else {
+                    rv = r4[x];
+                    rv = make_float4(rv.x / rZ, rv.y / rZ, rv.z / rZ, rv.w / rZ);
+                }
+                const float4 w = make_float4(fmaxf(rv.x - qv.x, 0.f), fmaxf(rv.y - qv.y, 0.f),
+                                             fmaxf(rv.z - qv.z, 0.f), fmaxf(rv.w - qv.w, 0.f));
+                r4[x] = w;
+                part += (w.x + w.y) + (w.z + w.w);
+                const int d0 = lo + 4 * x;
+                if (dsib >= d0 && dsib < d0 + 4)
+                    S.slot[S.parity].rnext = dsib == d0 ? w.x : dsib == d0 + 1 ? w.y : dsib == d0 + 2 ? w.z : w.w;
+            }
+        } else {
+#pragma unroll 4
+            for (int x = tid; x < n; x += ACC_THREADS) {
+                const float r = from_p ? exp2f((__ldg(lrow + lo + x) - Mv) * c) / Sv : rbuf[x] / rZ;
+                const float w = fmaxf(r - __ldg(qrow + lo + x), 0.f);
+                rbuf[x] = w;
+                part += w;
+                if (lo + x == dsib) S.slot[S.parity].rnext = w;
+            }
         }
         part = warp_sum(part);
         if (lane == 0) S.red_f[warp] = part;
@@ -320,8 +348,21 @@ __global__ void __launch_bounds__(ACC_THREADS, 1) accept_kernel(const AcceptPara
         const bool from_p = S.r_is_p != 0;
         const float Mv = S.rowM[v];
         const float *lrow = lb + (size_t)v * rowV;
-        if (from_p)
-            for (int x = tid; x < n; x += ACC_THREADS) rbuf[x] = exp2f((__ldg(lrow + lo + x) - Mv) * c);
+        if (from_p) {
+            if (VEC) {
+                const float4 *l4 = reinterpret_cast<const float4 *>(lrow + lo);
+                float4 *r4 = reinterpret_cast<float4 *>(rbuf);
+#pragma unroll 4
+                for (int x = tid; x < (n >> 2); x += ACC_THREADS) {
+                    const float4 lv = __ldg(l4 + x);
+                    r4[x] = make_float4(exp2f((lv.x - Mv) * c), exp2f((lv.y - Mv) * c), exp2f((lv.z - Mv) * c),
+                                        exp2f((lv.w - Mv) * c));
+                }
+            } else {
+#pragma unroll 4
+                for (int x = tid; x < n; x += ACC_THREADS) rbuf[x] = exp2f((__ldg(lrow + lo + x) - Mv) * c);
+            }
+        }
         __syncthreads();
         // contiguous segment per thread, summed in index order
         const int seg = (n + ACC_THREADS - 1) / ACC_THREADS;

@@ -64,13 +64,17 @@ SV_DEV int seq_tiles(const AttnParams &p, int b) {
     return ok ? (C + TILE_KEYS - 1) / TILE_KEYS : 0;
 }
 
-// Exclusive prefix of per-sequence tile counts into TP[0..B]; whole block participates.
-SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch) {
+// Exclusive prefix of per-sequence tile counts into TP[0..B] (and, when CL is
+// given, the context lengths into CL[0..B)); the whole block participates.
+SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch, int *CL = nullptr) {
     const int nt = blockDim.x, tid = threadIdx.x;
     const int per = (p.B + nt - 1) / nt;
     const int s0 = min(tid * per, p.B), s1 = min(s0 + per, p.B);
     int local = 0;
-    for (int b = s0; b < s1; ++b) local += seq_tiles(p, b);
+    for (int b = s0; b < s1; ++b) {
+        local += seq_tiles(p, b);
+        if (CL) CL[b] = p.ctx_lens[b];
+    }
     const int lane = tid & 31, warp = tid >> 5;
     int incl = local;
 #pragma unroll
@@ -121,8 +125,8 @@ SV_DEV TileInfo decode_tile(const int *TP, int B, int ups, int t) {
 constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle column of a tile
 
 struct TcLayout {
-    uint32_t stage_bytes, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_red, off_ms, off_as, off_lred,
-        off_misc, total;
+    uint32_t stage_bytes, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
+        off_lred, off_misc, total;
 };
 
 __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, int B) {
@@ -137,7 +141,8 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, in
     L.off_bar = L.off_p + NP * L.p_bytes;
     const int nbar = 2 * NST + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ + 2 /*wg*/;
     L.off_tp = L.off_bar + 8u * nbar;
-    L.off_red = (L.off_tp + 4u * (B + 1) + 15u) & ~15u;
+    L.off_cl = L.off_tp + 4u * (B + 1);
+    L.off_red = (L.off_cl + 4u * B + 15u) & ~15u;
     L.off_ms = L.off_red + 4u * 2 * 2 * 4 * RPh;   // [par][wg][warp][RPh]
     L.off_as = L.off_ms + 4u * 2 * RP;             // [par][RP]
     L.off_lred = L.off_as + 4u * 2 * RP;           // [par][RP]
@@ -178,6 +183,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     uint64_t *done_bar = o_empty + 2;
     uint64_t *wg_bar = done_bar + 1;  // warpgroup-local barriers of the two math warpgroups
     int *TP = reinterpret_cast<int *>(base + L.off_tp);
+    int *CL = reinterpret_cast<int *>(base + L.off_cl);
     float *red = reinterpret_cast<float *>(base + L.off_red);
     float *mS = reinterpret_cast<float *>(base + L.off_ms);
     float *aS = reinterpret_cast<float *>(base + L.off_as);
@@ -215,7 +221,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
         for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += TC_THREADS) q4[e] = make_uint4(0, 0, 0, 0);
     }
-    tile_prefix(p, TP, scratch);  // contains __syncthreads
+    tile_prefix(p, TP, scratch, CL);  // contains __syncthreads
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
@@ -251,19 +257,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         tma_load_3d(qdst + a * RP * 128, &P.tm_q, &q_full[qb], a * 64, h * p.G,
                                     ti.b * p.N + rc * P.Nc);
                 }
+                // gather the tile's page ids first (independent loads), then wait for the stage
+                const int C = CL[ti.b];
+                int blks[TILE_KEYS / PAGE];
+#pragma unroll
+                for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
+                    const int page = ti.j * (TILE_KEYS / PAGE) + pg;
+                    blks[pg] = page * PAGE < C ? __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page) : -1;
+                }
                 const int s = lt % NST;
                 if (!mbar_wait(&kv_empty[s], ((lt / NST) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
                 mbar_arrive_expect_tx(&kv_full[s], L.stage_bytes);
                 uint8_t *vdst = base + s * L.stage_bytes;
                 uint8_t *kdst = vdst + nDA * ATOM;
-                const int C = __ldg(p.ctx_lens + ti.b);
+#pragma unroll
                 for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
-                    const int page = ti.j * (TILE_KEYS / PAGE) + pg;
-                    int blk = p.num_blocks;  // out of range: the TMA unit fills zeros
-                    if (page * PAGE < C) {
-                        const int x = __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page);
-                        if (x >= 0 && x < p.num_blocks) blk = x;
-                    }
+                    // out of range (or past ctx_len): a coordinate past the pool, which the TMA unit fills with zeros
+                    const int blk = (blks[pg] >= 0 && blks[pg] < p.num_blocks) ? blks[pg] : p.num_blocks;
                     for (int a = 0; a < nDA; ++a) {
                         tma_load_4d(vdst + a * ATOM + pg * 2048, &P.tm_v, &kv_full[s], a * 64, 0, h, blk);
                         tma_load_4d(kdst + a * ATOM + pg * 2048, &P.tm_k, &kv_full[s], a * 64, 0, h, blk);
@@ -416,7 +426,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                 ub = ti.b;
                 uh = ti.hr / p.RC;
                 urc = ti.hr - uh * p.RC;
-                uC = __ldg(p.ctx_lens + ub);
+                uC = CL[ub];
                 urows = min(p.rows_unit, p.R - urc * p.rows_unit);
             }
             // ---- softmax of tile lt ----
@@ -448,8 +458,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
 #pragma unroll
             for (int c = 0; c < RPh; ++c) {
-                const float m = warp_max(sv[c]);
-                if (lane == 0) rd[c] = m;
+                float m;
+                asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(sv[c]));
+                if (lane == (c & 31)) rd[c] = m;
             }
             if (!(ok = wg_sync())) break;
             if (wiw == 0) {

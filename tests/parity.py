@@ -6,7 +6,9 @@ Accept: greedy results must match bit for bit. With sampling, a decision may
 differ only where the oracle marked a near tie (|u - r(d)/q(d)| < 1e-5 for an
 accept test, or a draw threshold within 1e-5 of a CDF step); everything after
 the first near tie of a sequence is then exempt, and the number of exempt
-sequences is reported.
+sequences is reported. An exempt draw must still pick a token inside the
+oracle's band: a token the draw selects for some threshold within 1e-5 of
+the total mass of the sampled one.
 """
 from __future__ import annotations
 
@@ -69,6 +71,9 @@ def compare_accept(gpu_len, gpu_next, gpu_path, gpu_status, orc, greedy: bool):
             continue
         if tw:
             exempt += 1
+            if not (orc.draw_lo[b] <= gpu_next[b] <= orc.draw_hi[b]):
+                bad.append((b, f"near-tie draw {int(gpu_next[b])} outside [{int(orc.draw_lo[b])}, "
+                               f"{int(orc.draw_hi[b])}]"))
             continue
         if gpu_next[b] != orc.next_token[b]:
             bad.append((b, f"next_token {int(gpu_next[b])} != {int(orc.next_token[b])}"))

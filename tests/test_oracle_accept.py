@@ -254,3 +254,12 @@ def test_flags_for_bad_inputs():
     assert r.flags.tolist()[0] == 1 and r.accept_len[0] == 0 and r.next_token[0] == 0
     assert r.flags[1] & 4 and r.accept_len[1] == 0
     assert r.flags[2] == 0
+
+
+def test_draw_band_brackets_the_drawn_token():
+    a = W.make_accept_inputs(200, 5, 3000, seed=12, logit_std=3.0, draft_noise=0.75, temperature=1.0)
+    r = oracle.accept(a.target_logits, a.draft_probs, a.draft_tokens, 1.0, seed=4)
+    assert (r.draw_lo <= r.next_token).all() and (r.next_token <= r.draw_hi).all()
+    # the band is a single token unless the draw is a near tie
+    narrow = r.draw_lo == r.draw_hi
+    assert (narrow | (r.tie_draw > 0) | (r.tie_depth >= 0)).all()
