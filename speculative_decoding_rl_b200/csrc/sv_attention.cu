@@ -52,7 +52,8 @@ namespace sv {
 using namespace tc;
 
 constexpr int TC_THREADS = 320;
-constexpr int MATH_THREADS_PER_WG = 128;
+constexpr int MATH_WARPS = 8;        // warps 2..9; each arrives once (lane 0 after __syncwarp)
+constexpr int WARPS_PER_WG = 4;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
 
 // ---------------------------------------------------------------------------
@@ -126,7 +127,7 @@ constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle colu
 
 struct TcLayout {
     uint32_t stage_bytes, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
-        off_lred, off_misc, total;
+        off_lred, off_rowi, off_umask, off_misc, total;
 };
 
 __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, int B) {
@@ -146,7 +147,9 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, in
     L.off_ms = L.off_red + 4u * 2 * 2 * 4 * RPh;   // [par][wg][warp][RPh]
     L.off_as = L.off_ms + 4u * 2 * RP;             // [par][RP]
     L.off_lred = L.off_as + 4u * 2 * RP;           // [par][RP]
-    L.off_misc = L.off_lred + 4u * 2 * 4 * RPh;    // [wg][warp][RPh]
+    L.off_rowi = L.off_lred + 4u * 2 * 4 * RPh;    // [wg][warp][RPh]
+    L.off_umask = (L.off_rowi + 4u * RP + 15u) & ~15u;  // row r -> query row offset r / G
+    L.off_misc = L.off_umask + 8u * 2 * 64;        // [wg][64] draft-mask words of the current unit
     L.total = L.off_misc + 64u;
     return L;
 }
@@ -188,6 +191,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     float *mS = reinterpret_cast<float *>(base + L.off_ms);
     float *aS = reinterpret_cast<float *>(base + L.off_as);
     float *lred = reinterpret_cast<float *>(base + L.off_lred);
+    int *rowi = reinterpret_cast<int *>(base + L.off_rowi);
+    uint64_t *umask = reinterpret_cast<uint64_t *>(base + L.off_umask);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
     int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // 10 ints, used once
@@ -198,13 +203,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         for (int s = 0; s < NST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
-            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 2 * MATH_THREADS_PER_WG);
-            mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], 2 * MATH_THREADS_PER_WG);
+            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], MATH_WARPS);
+            mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], MATH_WARPS);
         }
-        for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], 2 * MATH_THREADS_PER_WG); mbar_init(&p_empty[i], 1); }
+        for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], MATH_WARPS); mbar_init(&p_empty[i], 1); }
         mbar_init(done_bar, 1);
-        mbar_init(&wg_bar[0], MATH_THREADS_PER_WG);
-        mbar_init(&wg_bar[1], MATH_THREADS_PER_WG);
+        mbar_init(&wg_bar[0], WARPS_PER_WG);
+        mbar_init(&wg_bar[1], WARPS_PER_WG);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -217,6 +222,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         tma_prefetch_desc(&P.tm_v);
         tma_prefetch_desc(&P.tm_q);
     }
+    for (int r = tid; r < RP; r += TC_THREADS) rowi[r] = r / p.G;
     {  // zero both query buffers: rows past a unit's real rows stay zero
         uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
         for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += TC_THREADS) q4[e] = make_uint4(0, 0, 0, 0);
@@ -292,53 +298,73 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         }
     } else if (warp == 1) {
         // -------------------------- MMA issuer ----------------------------
+        // Polls both queues and issues whichever product is ready: QK of the
+        // next tile once its K stage, its query rows and an S buffer are
+        // ready; PV of the oldest softmaxed tile once its P and an O buffer
+        // are ready. Neither waits behind the other.
         if (lane == 0) {
             constexpr uint32_t idq = idesc_bf16(128, RP, false, false);
             constexpr uint32_t idp = idesc_bf16(128, RP, true, true);
-            int lu = -1, qb = 0;
-            bool ok = true;
-            auto issue_pv = [&](int jt) -> bool {
-                const int s = jt % NST, pb = jt % NP, ob = jt & 1;
-                if (!mbar_wait(&p_full[pb], (jt / NP) & 1, abort_flag, WAIT_LIMIT_NS)) return false;
-                if (!mbar_wait(&o_empty[ob], ((jt >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) return false;
-                tc_fence_after();
-                const uint32_t va = smem_u32(base + s * L.stage_bytes);
-                const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
+            int nq = 0, np = 0, lu = -1, qb = 0;
+            TileInfo tq = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+            uint32_t idle = 0;
+            uint64_t idle_since = 0;
+            while (np < ntiles) {
+                bool progressed = false;
+                if (nq < ntiles) {
+                    const bool newu = (nq == 0 || tq.j == 0);
+                    const int lu_n = newu ? lu + 1 : lu;
+                    const int qb_n = lu_n & 1;
+                    const int s = nq % NST, sb = nq & 1;
+                    if ((!newu || mbar_test(&q_full[qb_n], (lu_n >> 1) & 1)) &&
+                        mbar_test(&kv_full[s], (nq / NST) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
+                        lu = lu_n;
+                        qb = qb_n;
+                        tc_fence_after();
+                        const uint32_t ka = smem_u32(base + s * L.stage_bytes + nDA * ATOM);
+                        const uint32_t qa = smem_u32(base + L.off_q + qb * L.q_bytes);
 #pragma unroll
-                for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(va + kk * 2048, ATOM, 1024);
-                    const uint64_t bd = sw128_desc(pa + kk * 2048, ATOM, 1024);
-                    mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, kk > 0);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(ka + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
+                            const uint64_t bd = sw128_desc(qa + (kk >> 2) * (RP * 128) + (kk & 3) * 32, 16, 1024);
+                            mma_bf16_ss(tmem + sb * RPa, ad, bd, idq, kk > 0);
+                        }
+                        mma_commit(&s_full[sb]);
+                        if (nq == ntiles - 1 || tq.j == tq.Tb - 1) mma_commit(&q_empty[qb]);
+                        ++nq;
+                        if (nq < ntiles) tq = decode_tile(TP, p.B, ups, t_begin + nq);
+                        progressed = true;
+                    }
                 }
-                mma_commit(&o_full[ob]);
-                mma_commit(&p_empty[pb]);
-                mma_commit(&kv_empty[s]);
-                return true;
-            };
-            for (int lt = 0; lt < ntiles && ok; ++lt) {
-                const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
-                const int s = lt % NST, sb = lt & 1;
-                if (lt == 0 || ti.j == 0) {
-                    ++lu;
-                    qb = lu & 1;
-                    if (!mbar_wait(&q_full[qb], (lu >> 1) & 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
-                }
-                if (!mbar_wait(&kv_full[s], (lt / NST) & 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
-                if (!mbar_wait(&s_empty[sb], ((lt >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) { ok = false; break; }
-                tc_fence_after();
-                const uint32_t ka = smem_u32(base + s * L.stage_bytes + nDA * ATOM);
-                const uint32_t qa = smem_u32(base + L.off_q + qb * L.q_bytes);
+                if (np < nq) {
+                    const int s = np % NST, pb = np % NP, ob = np & 1;
+                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&o_empty[ob], ((np >> 1) & 1) ^ 1)) {
+                        tc_fence_after();
+                        const uint32_t va = smem_u32(base + s * L.stage_bytes);
+                        const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t ad = sw128_desc(ka + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = sw128_desc(qa + (kk >> 2) * (RP * 128) + (kk & 3) * 32, 16, 1024);
-                    mma_bf16_ss(tmem + sb * RPa, ad, bd, idq, kk > 0);
+                        for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
+                            const uint64_t ad = sw128_desc(va + kk * 2048, ATOM, 1024);
+                            const uint64_t bd = sw128_desc(pa + kk * 2048, ATOM, 1024);
+                            mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, kk > 0);
+                        }
+                        mma_commit(&o_full[ob]);
+                        mma_commit(&p_empty[pb]);
+                        mma_commit(&kv_empty[s]);
+                        ++np;
+                        progressed = true;
+                    }
                 }
-                mma_commit(&s_full[sb]);
-                if (lt == ntiles - 1 || ti.j == ti.Tb - 1) mma_commit(&q_empty[qb]);
-                if (lt > 0) ok = issue_pv(lt - 1);
+                if (progressed) {
+                    idle = 0;
+                } else if (++idle > 8 && (__nanosleep(20), (idle & 63) == 0)) {
+                    // bounded like every other wait: give up after the limit without progress
+                    if (*abort_flag) break;
+                    const uint64_t now = globaltimer_ns();
+                    if (idle == 64) idle_since = now;
+                    else if (now - idle_since > WAIT_LIMIT_NS) { *abort_flag = 1; break; }
+                }
             }
-            if (ok && ntiles > 0) issue_pv(ntiles - 1);
             mma_commit(done_bar);  // every MMA of this CTA has finished before TMEM is freed
             mbar_wait_time(done_bar, 0, WAIT_LIMIT_NS);
         }
@@ -360,6 +386,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         int cur_u = -1, last_par = 0;
         int ub = 0, uh = 0, urc = 0, uC = 0, urows = 0;
 
+        // one arrival per warp: every lane's prior work is ordered by __syncwarp
+        auto warp_arrive = [&](uint64_t *b) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(b);
+        };
         // warp-uniform bounded wait: the tcgen05 loads that follow are .sync.aligned
         auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
             const bool r = mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
@@ -373,14 +404,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             tmem_ld_cols<RPh>(lane_base + (2 + ob) * RPa + col0, o);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&o_empty[ob]);
-            const float *al = aS + (jt & 1) * RP + col0;
+            warp_arrive(&o_empty[ob]);
+            const float4 *al4 = reinterpret_cast<const float4 *>(aS + (jt & 1) * RP + col0);
 #pragma unroll
-            for (int c = 0; c < RPh; ++c) acc[c] = fmaf(acc[c], al[c], o[c]);
+            for (int c4 = 0; c4 < RPh / 4; ++c4) {
+                const float4 a4 = al4[c4];
+                acc[c4 * 4 + 0] = fmaf(acc[c4 * 4 + 0], a4.x, o[c4 * 4 + 0]);
+                acc[c4 * 4 + 1] = fmaf(acc[c4 * 4 + 1], a4.y, o[c4 * 4 + 1]);
+                acc[c4 * 4 + 2] = fmaf(acc[c4 * 4 + 2], a4.z, o[c4 * 4 + 2]);
+                acc[c4 * 4 + 3] = fmaf(acc[c4 * 4 + 3], a4.w, o[c4 * 4 + 3]);
+            }
             return true;
         };
         auto wg_sync = [&]() -> bool {
-            mbar_arrive(&wg_bar[wg]);
+            warp_arrive(&wg_bar[wg]);
             const bool r = wait_w(&wg_bar[wg], wg_phase);
             wg_phase ^= 1;
             return r;
@@ -428,6 +465,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                 urc = ti.hr - uh * p.RC;
                 uC = CL[ub];
                 urows = min(p.rows_unit, p.R - urc * p.rows_unit);
+                if (p.mask) {
+                    for (int k = wiw * 32 + lane; k < p.N; k += 128)
+                        umask[wg * 64 + k] = __ldg(p.mask + (size_t)ub * p.N + k);
+                    if (!(ok = wg_sync())) break;
+                }
             }
             // ---- softmax of tile lt ----
             const int sb = lt & 1, par = lt & 1;
@@ -437,23 +479,25 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             tmem_ld_cols<RPh>(lane_base + sb * RPa + col0, sv);
             tmem_wait_ld();
             tc_fence_before();
-            mbar_arrive(&s_empty[sb]);
+            warp_arrive(&s_empty[sb]);
 
+            // Scores stay unscaled here: the 1/sqrt(D) * log2(e) factor is positive,
+            // so it is applied to the column maximum and folded into the exponent.
             const int key = ti.j * TILE_KEYS + ell;
             const bool valid = key < uC;
             const int newk = key - (uC - p.N);
+            if (__any_sync(0xffffffffu, !valid || newk >= 0)) {
+                // tile holds keys past ctx_len or new (masked) keys: per-element visibility
+                const int ibase = urc * P.Nc;
 #pragma unroll
-            for (int c = 0; c < RPh; ++c) {
-                float v = sv[c] * p.scale_log2;
-                if (!valid) {
-                    v = -INFINITY;
-                } else if (newk >= 0 && col0 + c < urows) {
-                    const int i = urc * P.Nc + (col0 + c) / p.G;
-                    const bool vis = p.mask ? ((__ldg(p.mask + (size_t)ub * p.N + i) >> newk) & 1ull) != 0
-                                            : newk <= i;
-                    if (!vis) v = -INFINITY;
+                for (int c = 0; c < RPh; ++c) {
+                    bool vis = valid;
+                    if (valid && newk >= 0 && col0 + c < urows) {
+                        const int i = ibase + rowi[col0 + c];
+                        vis = p.mask ? ((umask[wg * 64 + i] >> newk) & 1ull) != 0 : newk <= i;
+                    }
+                    if (!vis) sv[c] = -INFINITY;
                 }
-                sv[c] = v;
             }
             float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
 #pragma unroll
@@ -466,26 +510,35 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             if (wiw == 0) {
                 for (int c = lane; c < RPh; c += 32) {
                     const float mo = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
-                    float mx = mo;
-                    for (int w = 0; w < 4; ++w) mx = fmaxf(mx, red[((par * 2 + wg) * 4 + w) * RPh + c]);
+                    float rmax = -INFINITY;
+                    for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * 2 + wg) * 4 + w) * RPh + c]);
+                    const float mx = fmaxf(mo, rmax * p.scale_log2);
                     mS[par * RP + col0 + c] = mx;
-                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : exp2f(mo - mx);
+                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(mo - mx);
                 }
             }
             if (!(ok = wg_sync())) break;
             last_par = par;
-            const float *ms = mS + par * RP + col0;
-            const float *as = aS + par * RP + col0;
+            const float4 *ms4 = reinterpret_cast<const float4 *>(mS + par * RP + col0);
+            const float4 *as4 = reinterpret_cast<const float4 *>(aS + par * RP + col0);
+            const float sc = p.scale_log2;
             uint32_t packed[RPh / 2];
 #pragma unroll
-            for (int c = 0; c < RPh; c += 2) {
-                const float m0 = ms[c], m1 = ms[c + 1];
-                const float p0 = (m0 == -INFINITY) ? 0.f : exp2f(sv[c] - m0);
-                const float p1 = (m1 == -INFINITY) ? 0.f : exp2f(sv[c + 1] - m1);
-                lsum[c] = fmaf(lsum[c], as[c], p0);
-                lsum[c + 1] = fmaf(lsum[c + 1], as[c + 1], p1);
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                packed[c / 2] = *reinterpret_cast<uint32_t *>(&h2);
+            for (int c4 = 0; c4 < RPh / 4; ++c4) {
+                const float4 m4 = ms4[c4], a4 = as4[c4];
+                const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                float pp[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int c = c4 * 4 + k;
+                    // p = 2^(s*scale - m); a column with no visible key yet (m = -inf) gives 0
+                    pp[k] = mm[k] == -INFINITY ? 0.f : ex2_approx(fmaf(sv[c], sc, -mm[k]));
+                    lsum[c] = fmaf(lsum[c], aa[k], pp[k]);
+                }
+                __nv_bfloat162 h0 = __floats2bfloat162_rn(pp[0], pp[1]);
+                __nv_bfloat162 h1 = __floats2bfloat162_rn(pp[2], pp[3]);
+                packed[c4 * 2] = *reinterpret_cast<uint32_t *>(&h0);
+                packed[c4 * 2 + 1] = *reinterpret_cast<uint32_t *>(&h1);
             }
             const int pb = lt % NP;
             if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
@@ -506,7 +559,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&p_full[pb]);
+            warp_arrive(&p_full[pb]);
             // ---- rescale-and-add the previous tile of the same unit ----
             if (!first)
                 if (!(ok = correction(lt - 1))) break;

@@ -52,6 +52,19 @@ SV_DEV bool mbar_try_wait(uint64_t *b, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test of a phase (for polling several barriers).
+SV_DEV bool mbar_test(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait: gives up after `limit_ns` of wall time, or as soon as another
 // thread of the CTA has raised *abort; on giving up it raises *abort and
 // returns false. Every wait in the attention kernel goes through here.
@@ -79,6 +92,13 @@ SV_DEV bool mbar_wait_time(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
         if (mbar_try_wait(b, parity)) return true;
         if ((i & 63) == 0 && globaltimer_ns() - t0 > limit_ns) return false;
     }
+}
+
+// 2^x on the SFU (ex2.approx.ftz: relative error about 2^-22; 2^-inf = 0).
+SV_DEV float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // ------------------------------- fences ------------------------------------
