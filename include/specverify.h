@@ -86,7 +86,7 @@ typedef enum {
  * t < ctx_len - N. Scores are q.k / sqrt(D); out = softmax(scores) . V,
  * accumulated in fp32 (P is rounded to bf16 for the P.V tensor-core product).
  * Limits: 1 <= N <= 64, D in {64, 128}, block_size 16, Hq % Hkv == 0,
- * Hq/Hkv <= 96, B <= 1024. q, out and the pools must be 16-byte aligned.
+ * Hq/Hkv <= 96, B <= 512. q, out and the pools must be 16-byte aligned.
  * A sequence flagged SV_FLAG_BAD_CONTEXT gets out = 0; one flagged
  * SV_FLAG_BAD_BLOCK reads zeros for the bad pages. A row that sees no key
  * gets out = 0.

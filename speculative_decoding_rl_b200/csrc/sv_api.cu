@@ -31,7 +31,7 @@ sv_status check_attn_desc(const sv_attn_desc *d) {
     if (d->block_size != sv::PAGE) return fail(SV_ERR_UNSUPPORTED, "block_size must be 16");
     if (d->max_blocks_per_seq < 1) return fail(SV_ERR_INVALID_ARG, "max_blocks_per_seq < 1");
     if (d->num_blocks < 1) return fail(SV_ERR_INVALID_ARG, "num_blocks < 1");
-    if (d->num_seqs > sv::MAX_SEQS) return fail(SV_ERR_UNSUPPORTED, "num_seqs > 1024");
+    if (d->num_seqs > sv::MAX_SEQS) return fail(SV_ERR_UNSUPPORTED, "num_seqs > 512");
     if (d->num_q_heads / d->num_kv_heads > sv::ROWS_MAX)
         return fail(SV_ERR_UNSUPPORTED, "more than 96 query heads per KV head");
     if ((long long)d->max_blocks_per_seq * sv::PAGE > (1LL << 30)) return fail(SV_ERR_UNSUPPORTED, "context too long");

@@ -51,7 +51,7 @@ namespace sv {
 
 using namespace tc;
 
-constexpr int TC_THREADS = 320;
+constexpr int TC_THREADS = 352;  // warps 0 (K/Q loads), 1 (MMA), 2-9 (softmax), 10 (V loads)
 constexpr int MATH_WARPS = 8;        // warps 2..9; each arrives once (lane 0 after __syncwarp)
 constexpr int WARPS_PER_WG = 4;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
@@ -126,21 +126,24 @@ SV_DEV TileInfo decode_tile(const int *TP, int B, int ups, int t) {
 constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle column of a tile
 
 struct TcLayout {
-    uint32_t stage_bytes, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
-        off_lred, off_rowi, off_umask, off_misc, total;
+    uint32_t tile_bytes, off_k, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
+        off_lred, off_rowi, off_umask, off_vote, off_misc, total;
 };
 
-__host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, int B) {
+// V ring first (slots 0..NV-1), then the K ring: a V slot plus 16 KB is always
+// inside the allocation (the D = 64 PV product reads one unused atom there).
+__host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int NP, int B) {
     TcLayout L;
     const int nDA = D / 64;
     const int RPh = RP / 2;
-    L.stage_bytes = 2u * nDA * ATOM;
-    L.off_q = NST * L.stage_bytes;
+    L.tile_bytes = (uint32_t)nDA * ATOM;  // 128 keys of K or of V
+    L.off_k = NV * L.tile_bytes;
+    L.off_q = L.off_k + NK * L.tile_bytes;
     L.q_bytes = (uint32_t)nDA * RP * 128u;
     L.off_p = L.off_q + 2u * L.q_bytes;
     L.p_bytes = (uint32_t)((RP + 63) / 64) * ATOM;
     L.off_bar = L.off_p + NP * L.p_bytes;
-    const int nbar = 2 * NST + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ + 2 /*wg*/;
+    const int nbar = 2 * NK + 2 * NV + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ + 2 /*wg*/;
     L.off_tp = L.off_bar + 8u * nbar;
     L.off_cl = L.off_tp + 4u * (B + 1);
     L.off_red = (L.off_cl + 4u * B + 15u) & ~15u;
@@ -149,7 +152,8 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NST, int NP, in
     L.off_lred = L.off_as + 4u * 2 * RP;           // [par][RP]
     L.off_rowi = L.off_lred + 4u * 2 * 4 * RPh;    // [wg][warp][RPh]
     L.off_umask = (L.off_rowi + 4u * RP + 15u) & ~15u;  // row r -> query row offset r / G
-    L.off_misc = L.off_umask + 8u * 2 * 64;        // [wg][64] draft-mask words of the current unit
+    L.off_vote = L.off_umask + 8u * 2 * 64;        // [wg][64] draft-mask words of the current unit
+    L.off_misc = L.off_vote + 4u * 2 * 2 * 4;      // [par][wg][warp] rescale votes
     L.total = L.off_misc + 64u;
     return L;
 }
@@ -159,7 +163,7 @@ struct TcParams {
     CUtensorMap tm_v;
     CUtensorMap tm_q;
     AttnParams a;
-    int NST, NP, Nc;
+    int NK, NV, NP, Nc;
     uint32_t epoch;
 };
 
@@ -172,14 +176,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     constexpr int RPh = RP / 2;
     constexpr int RPa = (RP + 31) / 32 * 32;  // TMEM columns per S / O buffer
     const AttnParams &p = P.a;
-    const int NST = P.NST, NP = P.NP;
+    const int NK = P.NK, NV = P.NV, NP = P.NP;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const TcLayout L = tc_layout(D, RP, NST, NP, p.B);
+    const TcLayout L = tc_layout(D, RP, NK, NV, NP, p.B);
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + L.off_bar);
-    uint64_t *kv_full = bar, *kv_empty = bar + NST;
-    uint64_t *q_full = bar + 2 * NST, *q_empty = q_full + 2;
+    uint64_t *k_full = bar, *k_empty = bar + NK;
+    uint64_t *v_full = bar + 2 * NK, *v_empty = v_full + NV;
+    uint64_t *q_full = v_empty + NV, *q_empty = q_full + 2;
     uint64_t *s_full = q_empty + 2, *s_empty = s_full + 2;
     uint64_t *p_full = s_empty + 2, *p_empty = p_full + NP;
     uint64_t *o_full = p_empty + NP, *o_empty = o_full + 2;
@@ -193,6 +198,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     float *lred = reinterpret_cast<float *>(base + L.off_lred);
     int *rowi = reinterpret_cast<int *>(base + L.off_rowi);
     uint64_t *umask = reinterpret_cast<uint64_t *>(base + L.off_umask);
+    int *vote = reinterpret_cast<int *>(base + L.off_vote);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
     int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // 10 ints, used once
@@ -200,7 +206,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s < NST; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+        for (int s = 0; s < NK; ++s) { mbar_init(&k_full[s], 1); mbar_init(&k_empty[s], 1); }
+        for (int s = 0; s < NV; ++s) { mbar_init(&v_full[s], 1); mbar_init(&v_empty[s], 1); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], MATH_WARPS);
@@ -245,15 +252,21 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     const int t_end = min(t_begin + W, total);
     const int ntiles = t_end - t_begin;
 
-    if (warp == 0) {
-        // ------------------------- TMA producer ---------------------------
+    if (warp == 0 || warp == 10) {
+        // ----------------- TMA producers (warp 0: Q and K, warp 10: V) -----------------
         if (lane == 0) {
+            const bool is_k = warp == 0;
+            const int NR = is_k ? NK : NV;
+            uint64_t *full = is_k ? k_full : v_full;
+            uint64_t *empty = is_k ? k_empty : v_empty;
+            const CUtensorMap *tm = is_k ? &P.tm_k : &P.tm_v;
+            uint8_t *ring = base + (is_k ? L.off_k : 0u);
             const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
             int lu = -1, issued_tiles = 0;
             for (int lt = 0; lt < ntiles; ++lt) {
                 const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
                 const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
-                if (lt == 0 || ti.j == 0) {
+                if (is_k && (lt == 0 || ti.j == 0)) {
                     ++lu;
                     const int qb = lu & 1;
                     if (!mbar_wait(&q_empty[qb], ((lu >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
@@ -263,7 +276,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         tma_load_3d(qdst + a * RP * 128, &P.tm_q, &q_full[qb], a * 64, h * p.G,
                                     ti.b * p.N + rc * P.Nc);
                 }
-                // gather the tile's page ids first (independent loads), then wait for the stage
+                // gather the tile's page ids first (independent loads), then wait for the slot
                 const int C = CL[ti.b];
                 int blks[TILE_KEYS / PAGE];
 #pragma unroll
@@ -271,29 +284,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     const int page = ti.j * (TILE_KEYS / PAGE) + pg;
                     blks[pg] = page * PAGE < C ? __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page) : -1;
                 }
-                const int s = lt % NST;
-                if (!mbar_wait(&kv_empty[s], ((lt / NST) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
-                mbar_arrive_expect_tx(&kv_full[s], L.stage_bytes);
-                uint8_t *vdst = base + s * L.stage_bytes;
-                uint8_t *kdst = vdst + nDA * ATOM;
+                const int s = lt % NR;
+                if (!mbar_wait(&empty[s], ((lt / NR) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                mbar_arrive_expect_tx(&full[s], L.tile_bytes);
+                uint8_t *dst = ring + s * L.tile_bytes;
 #pragma unroll
                 for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
                     // out of range (or past ctx_len): a coordinate past the pool, which the TMA unit fills with zeros
                     const int blk = (blks[pg] >= 0 && blks[pg] < p.num_blocks) ? blks[pg] : p.num_blocks;
-                    for (int a = 0; a < nDA; ++a) {
-                        tma_load_4d(vdst + a * ATOM + pg * 2048, &P.tm_v, &kv_full[s], a * 64, 0, h, blk);
-                        tma_load_4d(kdst + a * ATOM + pg * 2048, &P.tm_k, &kv_full[s], a * 64, 0, h, blk);
-                    }
+                    for (int a = 0; a < nDA; ++a)
+                        tma_load_4d(dst + a * ATOM + pg * 2048, tm, &full[s], a * 64, 0, h, blk);
                 }
                 issued_tiles = lt + 1;
             }
             if (*abort_flag) {
                 // let this CTA's own copies land before it can exit: the last
-                // use of every stage and query buffer must have completed
-                for (int lt = max(0, issued_tiles - NST); lt < issued_tiles; ++lt)
-                    mbar_wait_time(&kv_full[lt % NST], (lt / NST) & 1, WAIT_LIMIT_NS);
-                for (int u = max(0, lu - 1); u <= lu; ++u)
-                    mbar_wait_time(&q_full[u & 1], (u >> 1) & 1, WAIT_LIMIT_NS);
+                // use of every slot and query buffer must have completed
+                for (int lt = max(0, issued_tiles - NR); lt < issued_tiles; ++lt)
+                    mbar_wait_time(&full[lt % NR], (lt / NR) & 1, WAIT_LIMIT_NS);
+                if (is_k)
+                    for (int u = max(0, lu - 1); u <= lu; ++u)
+                        mbar_wait_time(&q_full[u & 1], (u >> 1) & 1, WAIT_LIMIT_NS);
             }
         }
     } else if (warp == 1) {
@@ -315,13 +326,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     const bool newu = (nq == 0 || tq.j == 0);
                     const int lu_n = newu ? lu + 1 : lu;
                     const int qb_n = lu_n & 1;
-                    const int s = nq % NST, sb = nq & 1;
+                    const int s = nq % NK, sb = nq & 1;
                     if ((!newu || mbar_test(&q_full[qb_n], (lu_n >> 1) & 1)) &&
-                        mbar_test(&kv_full[s], (nq / NST) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
+                        mbar_test(&k_full[s], (nq / NK) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
                         lu = lu_n;
                         qb = qb_n;
                         tc_fence_after();
-                        const uint32_t ka = smem_u32(base + s * L.stage_bytes + nDA * ATOM);
+                        const uint32_t ka = smem_u32(base + L.off_k + s * L.tile_bytes);
                         const uint32_t qa = smem_u32(base + L.off_q + qb * L.q_bytes);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
@@ -330,6 +341,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                             mma_bf16_ss(tmem + sb * RPa, ad, bd, idq, kk > 0);
                         }
                         mma_commit(&s_full[sb]);
+                        mma_commit(&k_empty[s]);
                         if (nq == ntiles - 1 || tq.j == tq.Tb - 1) mma_commit(&q_empty[qb]);
                         ++nq;
                         if (nq < ntiles) tq = decode_tile(TP, p.B, ups, t_begin + nq);
@@ -337,10 +349,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     }
                 }
                 if (np < nq) {
-                    const int s = np % NST, pb = np % NP, ob = np & 1;
-                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&o_empty[ob], ((np >> 1) & 1) ^ 1)) {
+                    const int s = np % NV, pb = np % NP, ob = np & 1;
+                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&o_empty[ob], ((np >> 1) & 1) ^ 1) &&
+                        mbar_test(&v_full[s], (np / NV) & 1)) {
                         tc_fence_after();
-                        const uint32_t va = smem_u32(base + s * L.stage_bytes);
+                        const uint32_t va = smem_u32(base + s * L.tile_bytes);
                         const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
 #pragma unroll
                         for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
@@ -350,7 +363,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         }
                         mma_commit(&o_full[ob]);
                         mma_commit(&p_empty[pb]);
-                        mma_commit(&kv_empty[s]);
+                        mma_commit(&v_empty[s]);
                         ++np;
                         progressed = true;
                     }
@@ -393,7 +406,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         };
         // warp-uniform bounded wait: the tcgen05 loads that follow are .sync.aligned
         auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
-            const bool r = mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
+            const bool r = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
             return __all_sync(0xffffffffu, r);
         };
         auto correction = [&](int jt) -> bool {
@@ -499,33 +512,61 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     if (!vis) sv[c] = -INFINITY;
                 }
             }
-            float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
+            // Running maxima are only raised when a score exceeds its column's
+            // current maximum by more than 2^RESCALE_LOG2 (after a unit's first
+            // tile this is rare): p = 2^(s*scale - m) then stays below 2^8, and
+            // the tile is folded in with alpha = 1. Otherwise the column maxima
+            // of the tile are reduced over the 128 keys and the state rescaled.
+            constexpr float RESCALE_LOG2 = 8.f;
+            const float sc = p.scale_log2;
+            const float *mo = mS + (par ^ 1) * RP + col0;
+            bool need = first;
+            if (!first) {
 #pragma unroll
-            for (int c = 0; c < RPh; ++c) {
-                float m;
-                asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(sv[c]));
-                if (lane == (c & 31)) rd[c] = m;
+                for (int c = 0; c < RPh; ++c) need |= sv[c] * sc > mo[c] + RESCALE_LOG2;
             }
+            const bool wneed = __any_sync(0xffffffffu, need);
+            if (lane == 0) vote[(par * 2 + wg) * 4 + wiw] = wneed;
             if (!(ok = wg_sync())) break;
-            if (wiw == 0) {
+            const bool rescale = vote[(par * 2 + wg) * 4 + 0] | vote[(par * 2 + wg) * 4 + 1] |
+                                 vote[(par * 2 + wg) * 4 + 2] | vote[(par * 2 + wg) * 4 + 3];
+            if (rescale) {
+                float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
+#pragma unroll
+                for (int c = 0; c < RPh; ++c) {
+                    float m;
+                    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(sv[c]));
+                    if (lane == (c & 31)) rd[c] = m;
+                }
+                if (!(ok = wg_sync())) break;
+                if (wiw == 0) {
+                    for (int c = lane; c < RPh; c += 32) {
+                        const float m_old = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
+                        float rmax = -INFINITY;
+                        for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * 2 + wg) * 4 + w) * RPh + c]);
+                        const float mx = fmaxf(m_old, rmax * sc);
+                        mS[par * RP + col0 + c] = mx;
+                        aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(m_old - mx);
+                    }
+                }
+                if (!(ok = wg_sync())) break;
+            } else if (wiw == 0) {
+                // keep the maxima; the previous tile's state needs no rescale.
+                // Readers of these slots are past the next tile's first sync.
                 for (int c = lane; c < RPh; c += 32) {
-                    const float mo = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
-                    float rmax = -INFINITY;
-                    for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * 2 + wg) * 4 + w) * RPh + c]);
-                    const float mx = fmaxf(mo, rmax * p.scale_log2);
-                    mS[par * RP + col0 + c] = mx;
-                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(mo - mx);
+                    mS[par * RP + col0 + c] = mo[c];
+                    aS[par * RP + col0 + c] = 1.f;
                 }
             }
-            if (!(ok = wg_sync())) break;
             last_par = par;
-            const float4 *ms4 = reinterpret_cast<const float4 *>(mS + par * RP + col0);
-            const float4 *as4 = reinterpret_cast<const float4 *>(aS + par * RP + col0);
-            const float sc = p.scale_log2;
+            const float *msrc = rescale ? mS + par * RP + col0 : mo;
+            const float *asrc = aS + par * RP + col0;
+            const float4 *ms4 = reinterpret_cast<const float4 *>(msrc);
             uint32_t packed[RPh / 2];
 #pragma unroll
             for (int c4 = 0; c4 < RPh / 4; ++c4) {
-                const float4 m4 = ms4[c4], a4 = as4[c4];
+                const float4 m4 = ms4[c4];
+                const float4 a4 = rescale ? reinterpret_cast<const float4 *>(asrc)[c4] : make_float4(1.f, 1.f, 1.f, 1.f);
                 const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, aa[4] = {a4.x, a4.y, a4.z, a4.w};
                 float pp[4];
 #pragma unroll
@@ -551,9 +592,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                                                        (ell & 7) * 128 + ((chunk ^ (ell & 7)) << 4));
                 *dst = make_uint4(packed[c8 * 4], packed[c8 * 4 + 1], packed[c8 * 4 + 2], packed[c8 * 4 + 3]);
             }
+            if (__any_sync(0xffffffffu, !valid) && wg == 0) {
+                // a key past ctx_len: its V row may hold anything (NaN) and P = 0 does not
+                // cancel it, so the row is zeroed once the tile's V has landed
+                if (!(ok = wait_w(&v_full[lt % NV], (lt / NV) & 1))) break;
+            }
             if (!valid && wg == 0) {
-                // a key past ctx_len: its V row may hold anything (NaN) and P = 0 does not cancel it
-                uint8_t *vrow = base + (lt % NST) * L.stage_bytes + ell * 128;
+                uint8_t *vrow = base + (lt % NV) * L.tile_bytes + ell * 128;
                 for (int a = 0; a < nDA; ++a)
                     for (int q = 0; q < 8; ++q)
                         reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
@@ -585,8 +630,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
 // (row of a unit, unit), one thread per head dimension. The CTA of row 0 of
 // each sequence's first unit also writes that sequence's status flags.
 // ---------------------------------------------------------------------------
+constexpr int COMBINE_MAX_SEGS = 512;  // > num_ctas + 1 on any current GPU
+
 __global__ void attn_combine_kernel(const AttnParams p, uint32_t epoch) {
-    const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x;
+    const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
     const int D = p.D, RU = p.rows_unit;
     const int ups = p.Hkv * p.RC;
     const int b = u / ups, hr = u - b * ups;
@@ -599,23 +646,38 @@ __global__ void attn_combine_kernel(const AttnParams p, uint32_t epoch) {
     const int *TP = p.ws_plan + 2;
     const int Tb = TP[b + 1] - TP[b];
     const size_t slot_floats = (size_t)RU * D + 2 * RU;
+    __shared__ float sw[COMBINE_MAX_SEGS];
+    __shared__ float red_m[4], red_l[4];
     float res = 0.f;
     if (Tb > 0) {
         const int tpre = ups * TP[b] + hr * Tb;
-        const int first = tpre / W, last = (tpre + Tb - 1) / W;
-        float M = -INFINITY;
-        for (int c = first; c <= last; ++c)
-            M = fmaxf(M, p.ws_partial[(size_t)(u + c) * slot_floats + (size_t)RU * D + r]);
-        if (M > -INFINITY) {
-            float L = 0.f, acc = 0.f;
-            for (int c = first; c <= last; ++c) {
-                const float *slot = p.ws_partial + (size_t)(u + c) * slot_floats;
-                const float m = slot[(size_t)RU * D + r];
-                if (m == -INFINITY) continue;
-                const float w = exp2f(m - M);
-                L = fmaf(w, slot[(size_t)RU * D + RU + r], L);
-                acc = fmaf(w, slot[(size_t)r * D + d], acc);
-            }
+        const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
+        const float *seg0 = p.ws_partial + (size_t)(u + first) * slot_floats;
+        // the segments' (m, l) in parallel, one segment per thread
+        float m = -INFINITY;
+        for (int k = d; k < n; k += nt) m = fmaxf(m, seg0[(size_t)k * slot_floats + (size_t)RU * D + r]);
+        m = warp_max(m);
+        if ((d & 31) == 0) red_m[d >> 5] = m;
+        __syncthreads();
+        float M = red_m[0];
+        for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_m[w]);
+        float L = 0.f;
+        for (int k = d; k < n; k += nt) {
+            const float *sg = seg0 + (size_t)k * slot_floats;
+            const float mk = sg[(size_t)RU * D + r];
+            const float wk = (mk == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mk - M);
+            sw[k] = wk;
+            L = fmaf(wk, sg[(size_t)RU * D + RU + r], L);
+        }
+        L = warp_sum(L);
+        if ((d & 31) == 0) red_l[d >> 5] = L;
+        __syncthreads();
+        L = 0.f;
+        for (int w = 0; w < (nt + 31) / 32; ++w) L += red_l[w];
+        if (L > 0.f) {
+            float acc = 0.f;
+#pragma unroll 4
+            for (int k = 0; k < n; ++k) acc = fmaf(sw[k], seg0[(size_t)k * slot_floats + (size_t)r * D + d], acc);
             res = acc / L;
         }
     }
@@ -717,17 +779,18 @@ constexpr int SMEM_LIMIT = 227 * 1024;
 
 template <int D, int RP>
 static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
-    // two KV stages at D=128 (four at D=64), double-buffered P when it fits
-    int NST = D == 128 ? 2 : 4;
-    int NP = 2;
-    TcLayout L = tc_layout(D, RP, NST, NP, P.a.B);
-    if (L.total + 1024 > (uint32_t)SMEM_LIMIT) {
-        NP = 1;
-        L = tc_layout(D, RP, NST, NP, P.a.B);
+    // deepest K/V rings and P buffering that fit, in order of preference
+    static const int choices[][3] = {{3, 4, 2}, {2, 4, 2}, {2, 3, 2}, {2, 3, 1}, {2, 2, 2}, {2, 2, 1}};
+    TcLayout L;
+    int k = 0;
+    for (; k < 6; ++k) {
+        L = tc_layout(D, RP, choices[k][0], choices[k][1], choices[k][2], P.a.B);
+        if (L.total + 1024 <= (uint32_t)SMEM_LIMIT) break;
     }
-    if (L.total + 1024 > (uint32_t)SMEM_LIMIT) return cudaErrorInvalidConfiguration;
-    P.NST = NST;
-    P.NP = NP;
+    if (k == 6) return cudaErrorInvalidConfiguration;
+    P.NK = choices[k][0];
+    P.NV = choices[k][1];
+    P.NP = choices[k][2];
     const size_t smem = L.total + 1024;
     auto kfn = attn_tc_kernel<D, RP>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -38,7 +38,7 @@ cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream);
 constexpr int TILE_KEYS = 128;
 constexpr int PAGE = 16;
 constexpr int ROWS_MAX = 96;       // query rows (N*G) one unit carries
-constexpr int MAX_SEQS = 1024;
+constexpr int MAX_SEQS = 512;
 
 struct AttnParams {
     const uint16_t *q;         // bf16 bits [B][N][Hq][D]

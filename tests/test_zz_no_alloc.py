@@ -49,7 +49,7 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_refuses_requests_beyond_the_scratch():
     a = W.make_attention_inputs(5, 8, 2, 128, [64], seed=3)
     call = AttentionCall(a)
-    big = sv.SvAttnDesc(1024, 16, 64, 8, 128, 16, 8, a.num_blocks)
+    big = sv.SvAttnDesc(512, 16, 64, 8, 128, 16, 8, a.num_blocks)
     assert sv.sv_verify_attention_workspace_size(big) > sv.SV_NOALLOC_SCRATCH_BYTES
     with pytest.raises(sv.SvError) as e:
         sv.sv_verify_attention_noalloc(big, call.q, call.kv, call.block_table, call.ctx_lens, None,
