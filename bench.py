@@ -35,6 +35,7 @@ if ROOT not in sys.path:
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
+from speculative_decoding_rl_b200 import replicas as R  # noqa: E402
 from speculative_decoding_rl_b200 import workloads as W  # noqa: E402
 
 METRIC = "verify-steps/s & accepted tok/s at 1 B200; KV+logit HBM GB/s as % of peak"
@@ -148,42 +149,24 @@ class ClockSampler:
 
 
 def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    world, rank, local = R.env_ranks()
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
     if world > 1:
-        import datetime
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(local)
+        R.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     return world, rank, local
 
 
 def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+    R.barrier(world)
 
 
 def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    return R.max_over_ranks(x, world, device="cuda")
 
 
 def sum_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return R.sum_over_ranks(x, world, device="cuda")
 
 
 # ---------------------------------------------------------------------------

@@ -51,9 +51,12 @@ namespace sv {
 
 using namespace tc;
 
-constexpr int TC_THREADS = 352;  // warps 0 (K/Q loads), 1 (MMA), 2-9 (softmax), 10 (V loads)
-constexpr int MATH_WARPS = 8;        // warps 2..9; each arrives once (lane 0 after __syncwarp)
+// Softmax warpgroups: 4 warps each (one TMEM lane quadrant per warp), each
+// owning CW consecutive row columns; a unit's padded row count RP = CW * NWG.
+constexpr int CW = 16;
 constexpr int WARPS_PER_WG = 4;
+__host__ __device__ constexpr int tc_nwg(int RP) { return RP / CW; }
+__host__ __device__ constexpr int tc_threads(int RP) { return 32 * (WARPS_PER_WG * tc_nwg(RP) + 4); }
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
 
 // ---------------------------------------------------------------------------
@@ -106,6 +109,12 @@ SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
     return lo;
 }
 
+// Floats per workspace partial slot: O [rows][D], running max [rows], row sum
+// [rows], padded to 256 bytes so every slot (and every O row) is 16-byte aligned.
+__host__ __device__ inline size_t slot_stride(int rows_unit, int D) {
+    return ((size_t)rows_unit * D + 2 * (size_t)rows_unit + 63) & ~(size_t)63;
+}
+
 struct TileInfo {
     int b, hr, j, Tb;
 };
@@ -127,7 +136,7 @@ constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle colu
 
 struct TcLayout {
     uint32_t tile_bytes, off_k, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
-        off_lred, off_rowi, off_umask, off_vote, off_misc, total;
+        off_lred, off_rowi, off_umask, off_vote, off_fin, off_misc, total;
 };
 
 // V ring first (slots 0..NV-1), then the K ring: a V slot plus 16 KB is always
@@ -135,7 +144,7 @@ struct TcLayout {
 __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int NP, int B) {
     TcLayout L;
     const int nDA = D / 64;
-    const int RPh = RP / 2;
+    const int NWG = tc_nwg(RP);
     L.tile_bytes = (uint32_t)nDA * ATOM;  // 128 keys of K or of V
     L.off_k = NV * L.tile_bytes;
     L.off_q = L.off_k + NK * L.tile_bytes;
@@ -143,18 +152,20 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int
     L.off_p = L.off_q + 2u * L.q_bytes;
     L.p_bytes = (uint32_t)((RP + 63) / 64) * ATOM;
     L.off_bar = L.off_p + NP * L.p_bytes;
-    const int nbar = 2 * NK + 2 * NV + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ + 2 /*wg*/;
+    const int nbar = 2 * NK + 2 * NV + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ +
+                     NWG /*wg*/;
     L.off_tp = L.off_bar + 8u * nbar;
     L.off_cl = L.off_tp + 4u * (B + 1);
     L.off_red = (L.off_cl + 4u * B + 15u) & ~15u;
-    L.off_ms = L.off_red + 4u * 2 * 2 * 4 * RPh;   // [par][wg][warp][RPh]
-    L.off_as = L.off_ms + 4u * 2 * RP;             // [par][RP]
-    L.off_lred = L.off_as + 4u * 2 * RP;           // [par][RP]
-    L.off_rowi = L.off_lred + 4u * 2 * 4 * RPh;    // [wg][warp][RPh]
-    L.off_umask = (L.off_rowi + 4u * RP + 15u) & ~15u;  // row r -> query row offset r / G
-    L.off_vote = L.off_umask + 8u * 2 * 64;        // [wg][64] draft-mask words of the current unit
-    L.off_misc = L.off_vote + 4u * 2 * 2 * 4;      // [par][wg][warp] rescale votes
-    L.total = L.off_misc + 64u;
+    L.off_ms = L.off_red + 4u * 2 * NWG * WARPS_PER_WG * CW;  // [par][wg][warp][CW] tile column maxima
+    L.off_as = L.off_ms + 4u * 2 * RP;                        // [par][RP] running maxima
+    L.off_lred = L.off_as + 4u * 2 * RP;                      // [par][RP] rescale factors
+    L.off_rowi = L.off_lred + 4u * NWG * WARPS_PER_WG * CW;   // [wg][warp][CW] row-sum partials
+    L.off_umask = (L.off_rowi + 4u * RP + 15u) & ~15u;        // [RP] row r -> r / G
+    L.off_vote = L.off_umask + 8u * NWG * 64;                 // [wg][64] mask words of the unit
+    L.off_fin = L.off_vote + 4u * 2 * NWG * WARPS_PER_WG;     // [par][wg][warp] rescale votes
+    L.off_misc = L.off_fin + 4u * RP;                         // [RP] row sums of a finished unit
+    L.total = L.off_misc + 16u + 4u * 32;
     return L;
 }
 
@@ -171,10 +182,14 @@ struct TcParams {
 // The tcgen05 split-context kernel.
 // ---------------------------------------------------------------------------
 template <int D, int RP>
-__global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_constant__ TcParams P) {
+__global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid_constant__ TcParams P) {
     constexpr int nDA = D / 64;
-    constexpr int RPh = RP / 2;
+    constexpr int NWG = tc_nwg(RP);
+    constexpr int MATH_WARPS = WARPS_PER_WG * NWG;
+    constexpr int NTHREADS = tc_threads(RP);
     constexpr int RPa = (RP + 31) / 32 * 32;  // TMEM columns per S / O buffer
+    constexpr int WARP_K = MATH_WARPS, WARP_MMA = MATH_WARPS + 1, WARP_V = MATH_WARPS + 2,
+                  WARP_ST = MATH_WARPS + 3;
     const AttnParams &p = P.a;
     const int NK = P.NK, NV = P.NV, NP = P.NP;
 
@@ -187,9 +202,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     uint64_t *q_full = v_empty + NV, *q_empty = q_full + 2;
     uint64_t *s_full = q_empty + 2, *s_empty = s_full + 2;
     uint64_t *p_full = s_empty + 2, *p_empty = p_full + NP;
-    uint64_t *o_full = p_empty + NP, *o_empty = o_full + 2;
-    uint64_t *done_bar = o_empty + 2;
-    uint64_t *wg_bar = done_bar + 1;  // warpgroup-local barriers of the two math warpgroups
+    uint64_t *o_full = p_empty + NP;   // [2] by tile parity: the tile's PV has completed
+    uint64_t *o_free = o_full + 2;     // [2] by unit parity: the unit's O buffer has been read out
+    uint64_t *done_bar = o_free + 2;
+    uint64_t *wg_bar = done_bar + 1;   // [NWG] warpgroup-local barriers
     int *TP = reinterpret_cast<int *>(base + L.off_tp);
     int *CL = reinterpret_cast<int *>(base + L.off_cl);
     float *red = reinterpret_cast<float *>(base + L.off_red);
@@ -199,9 +215,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     int *rowi = reinterpret_cast<int *>(base + L.off_rowi);
     uint64_t *umask = reinterpret_cast<uint64_t *>(base + L.off_umask);
     int *vote = reinterpret_cast<int *>(base + L.off_vote);
+    float *lfin = reinterpret_cast<float *>(base + L.off_fin);  // [RP] row sums of the finished unit
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
-    int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // 10 ints, used once
+    int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // one int per warp (<= 28), used once
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -211,28 +228,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
         for (int i = 0; i < 2; ++i) {
             mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1);
             mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], MATH_WARPS);
-            mbar_init(&o_full[i], 1); mbar_init(&o_empty[i], MATH_WARPS);
+            mbar_init(&o_full[i], 1); mbar_init(&o_free[i], MATH_WARPS);
         }
         for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], MATH_WARPS); mbar_init(&p_empty[i], 1); }
         mbar_init(done_bar, 1);
-        mbar_init(&wg_bar[0], WARPS_PER_WG);
-        mbar_init(&wg_bar[1], WARPS_PER_WG);
+        for (int g = 0; g < NWG; ++g) mbar_init(&wg_bar[g], WARPS_PER_WG);
         *abort_flag = 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == WARP_MMA) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == WARP_K && lane == 0) {
         tma_prefetch_desc(&P.tm_k);
         tma_prefetch_desc(&P.tm_v);
         tma_prefetch_desc(&P.tm_q);
     }
-    for (int r = tid; r < RP; r += TC_THREADS) rowi[r] = r / p.G;
+    for (int r = tid; r < RP; r += NTHREADS) rowi[r] = r / p.G;
     {  // zero both query buffers: rows past a unit's real rows stay zero
         uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
-        for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += TC_THREADS) q4[e] = make_uint4(0, 0, 0, 0);
+        for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += NTHREADS) q4[e] = make_uint4(0, 0, 0, 0);
     }
     tile_prefix(p, TP, scratch, CL);  // contains __syncthreads
     fence_proxy_async_smem();
@@ -244,18 +260,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
     const int ups = p.Hkv * p.RC;
     const int total = ups * TP[p.B];
     const int W = total > 0 ? (total + p.num_ctas - 1) / p.num_ctas : 1;
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0) {  // the combine kernel's copy of the schedule
         if (tid == 0) { p.ws_plan[0] = W; p.ws_plan[1] = total; }
-        for (int b = tid; b <= p.B; b += TC_THREADS) p.ws_plan[2 + b] = TP[b];
+        for (int b = tid; b <= p.B; b += NTHREADS) p.ws_plan[2 + b] = TP[b];
     }
     const int t_begin = min((int)blockIdx.x * W, total);
     const int t_end = min(t_begin + W, total);
     const int ntiles = t_end - t_begin;
 
-    if (warp == 0 || warp == 10) {
-        // ----------------- TMA producers (warp 0: Q and K, warp 10: V) -----------------
+    if (warp == WARP_K || warp == WARP_V) {
+        // ------------------- TMA producers (Q and K; V) -------------------
         if (lane == 0) {
-            const bool is_k = warp == 0;
+            const bool is_k = warp == WARP_K;
             const int NR = is_k ? NK : NV;
             uint64_t *full = is_k ? k_full : v_full;
             uint64_t *empty = is_k ? k_empty : v_empty;
@@ -266,6 +282,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             for (int lt = 0; lt < ntiles; ++lt) {
                 const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
                 const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
+                // gather the tile's page ids first (independent loads), then wait for the slot
+                const int C = CL[ti.b];
+                int blks[TILE_KEYS / PAGE];
+#pragma unroll
+                for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
+                    const int page = ti.j * (TILE_KEYS / PAGE) + pg;
+                    blks[pg] = page * PAGE < C ? __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page) : -1;
+                }
                 if (is_k && (lt == 0 || ti.j == 0)) {
                     ++lu;
                     const int qb = lu & 1;
@@ -275,14 +299,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     for (int a = 0; a < nDA; ++a)
                         tma_load_3d(qdst + a * RP * 128, &P.tm_q, &q_full[qb], a * 64, h * p.G,
                                     ti.b * p.N + rc * P.Nc);
-                }
-                // gather the tile's page ids first (independent loads), then wait for the slot
-                const int C = CL[ti.b];
-                int blks[TILE_KEYS / PAGE];
-#pragma unroll
-                for (int pg = 0; pg < TILE_KEYS / PAGE; ++pg) {
-                    const int page = ti.j * (TILE_KEYS / PAGE) + pg;
-                    blks[pg] = page * PAGE < C ? __ldg(p.block_table + (size_t)ti.b * p.max_blocks + page) : -1;
                 }
                 const int s = lt % NR;
                 if (!mbar_wait(&empty[s], ((lt / NR) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
@@ -307,17 +323,41 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         mbar_wait_time(&q_full[u & 1], (u >> 1) & 1, WAIT_LIMIT_NS);
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == WARP_ST) {
+        // ---------------- per-sequence status (and invalid sequences) ----------------
+        // Sequence b is handled by CTA b mod num_ctas: a context outside
+        // [N, max_blocks*16] gets SV_FLAG_BAD_CONTEXT and a zero output; a valid
+        // one is scanned for block ids outside the pool (SV_FLAG_BAD_BLOCK).
+        for (int b = blockIdx.x; b < p.B; b += p.num_ctas) {
+            const int C = CL[b];
+            const bool ctx_ok = C >= p.N && C <= p.max_blocks * PAGE;
+            int bad = 0;
+            if (ctx_ok) {
+                for (int jb = lane; jb < (C + PAGE - 1) / PAGE; jb += 32) {
+                    const int blk = __ldg(p.block_table + (size_t)b * p.max_blocks + jb);
+                    bad |= (blk < 0 || blk >= p.num_blocks);
+                }
+            } else {
+                uint4 *o4 = reinterpret_cast<uint4 *>(p.out + (size_t)b * p.N * p.Hq * D);
+                for (int e = lane; e < p.N * p.Hq * D / 8; e += 32) o4[e] = make_uint4(0, 0, 0, 0);
+            }
+            bad = __any_sync(0xffffffffu, bad);
+            if (p.status && lane == 0)
+                p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0);
+        }
+    } else if (warp == WARP_MMA) {
         // -------------------------- MMA issuer ----------------------------
         // Polls both queues and issues whichever product is ready: QK of the
-        // next tile once its K stage, its query rows and an S buffer are
-        // ready; PV of the oldest softmaxed tile once its P and an O buffer
-        // are ready. Neither waits behind the other.
+        // next tile once its K slot, its query rows and an S buffer are ready;
+        // PV of the oldest softmaxed tile once its P and V are ready (and, at
+        // a unit's first tile, once the unit's O buffer has been read out).
+        // PV accumulates a unit's tiles in place in TMEM.
         if (lane == 0) {
             constexpr uint32_t idq = idesc_bf16(128, RP, false, false);
             constexpr uint32_t idp = idesc_bf16(128, RP, true, true);
-            int nq = 0, np = 0, lu = -1, qb = 0;
+            int nq = 0, np = 0, lu = -1, qb = 0, lup = -1;
             TileInfo tq = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+            TileInfo tp = tq;
             uint32_t idle = 0;
             uint64_t idle_since = 0;
             while (np < ntiles) {
@@ -349,9 +389,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     }
                 }
                 if (np < nq) {
-                    const int s = np % NV, pb = np % NP, ob = np & 1;
-                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&o_empty[ob], ((np >> 1) & 1) ^ 1) &&
-                        mbar_test(&v_full[s], (np / NV) & 1)) {
+                    const bool newu = (np == 0 || tp.j == 0);
+                    const int lup_n = newu ? lup + 1 : lup;
+                    const int s = np % NV, pb = np % NP, ob = lup_n & 1;
+                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&v_full[s], (np / NV) & 1) &&
+                        (!newu || mbar_test(&o_free[ob], ((lup_n >> 1) & 1) ^ 1))) {
+                        lup = lup_n;
                         tc_fence_after();
                         const uint32_t va = smem_u32(base + s * L.tile_bytes);
                         const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
@@ -359,12 +402,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                         for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
                             const uint64_t ad = sw128_desc(va + kk * 2048, ATOM, 1024);
                             const uint64_t bd = sw128_desc(pa + kk * 2048, ATOM, 1024);
-                            mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, kk > 0);
+                            mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, (kk > 0 || !newu) ? 1u : 0u);
                         }
-                        mma_commit(&o_full[ob]);
+                        mma_commit(&o_full[np & 1]);
                         mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[s]);
                         ++np;
+                        if (np < ntiles) tp = decode_tile(TP, p.B, ups, t_begin + np);
                         progressed = true;
                     }
                 }
@@ -382,21 +426,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             mbar_wait_time(done_bar, 0, WAIT_LIMIT_NS);
         }
     } else {
-        // ---------------------- softmax / correction ----------------------
-        const int wg = (warp - 2) >> 2;   // column half
-        const int wiw = (warp - 2) & 3;   // warp within the warpgroup
-        const int wq = warp & 3;          // TMEM lane quadrant this warp may access
-        const int ell = wq * 32 + lane;   // key (S) / head dim (O) lane
-        const int col0 = wg * RPh;
+        // ------------------------------ softmax ------------------------------
+        const int wg = warp >> 2;          // warpgroup: owns row columns [wg*CW, wg*CW + CW)
+        const int wiw = warp & 3;          // warp within the warpgroup = TMEM lane quadrant
+        const int ell = wiw * 32 + lane;   // key (S) / head dim (O) lane
+        const int col0 = wg * CW;
         uint32_t wg_phase = 0;
-        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-        float acc[RPh], lsum[RPh];
+        const uint32_t lane_base = tmem + ((uint32_t)(wiw * 32) << 16);
+        float lsum[CW];
 #pragma unroll
-        for (int c = 0; c < RPh; ++c) { acc[c] = 0.f; lsum[c] = 0.f; }
-        const size_t slot_floats = (size_t)p.rows_unit * D + 2 * p.rows_unit;
+        for (int c = 0; c < CW; ++c) lsum[c] = 0.f;
+        const size_t slot_floats = slot_stride(p.rows_unit, D);
         bool ok = true;
 
-        int cur_u = -1, last_par = 0;
+        int cur_u = -1, last_par = 0, lu = -1;
         int ub = 0, uh = 0, urc = 0, uC = 0, urows = 0;
 
         // one arrival per warp: every lane's prior work is ordered by __syncwarp
@@ -404,30 +447,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             __syncwarp();
             if (lane == 0) mbar_arrive(b);
         };
-        // warp-uniform bounded wait: the tcgen05 loads that follow are .sync.aligned
+        // warp-uniform bounded wait: the tcgen05 accesses that follow are .sync.aligned
         auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
             const bool r = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
             return __all_sync(0xffffffffu, r);
-        };
-        auto correction = [&](int jt) -> bool {
-            const int ob = jt & 1;
-            if (!wait_w(&o_full[ob], (jt >> 1) & 1)) return false;
-            tc_fence_after();
-            float o[RPh];
-            tmem_ld_cols<RPh>(lane_base + (2 + ob) * RPa + col0, o);
-            tmem_wait_ld();
-            tc_fence_before();
-            warp_arrive(&o_empty[ob]);
-            const float4 *al4 = reinterpret_cast<const float4 *>(aS + (jt & 1) * RP + col0);
-#pragma unroll
-            for (int c4 = 0; c4 < RPh / 4; ++c4) {
-                const float4 a4 = al4[c4];
-                acc[c4 * 4 + 0] = fmaf(acc[c4 * 4 + 0], a4.x, o[c4 * 4 + 0]);
-                acc[c4 * 4 + 1] = fmaf(acc[c4 * 4 + 1], a4.y, o[c4 * 4 + 1]);
-                acc[c4 * 4 + 2] = fmaf(acc[c4 * 4 + 2], a4.z, o[c4 * 4 + 2]);
-                acc[c4 * 4 + 3] = fmaf(acc[c4 * 4 + 3], a4.w, o[c4 * 4 + 3]);
-            }
-            return true;
         };
         auto wg_sync = [&]() -> bool {
             warp_arrive(&wg_bar[wg]);
@@ -435,32 +458,66 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             wg_phase ^= 1;
             return r;
         };
-        auto finalize = [&]() -> bool {
+        // output row r of the current unit -> element offset of (b, i, hq, 0) in out
+        auto out_row = [&](int r) -> size_t {
+            const int ridx = urc * p.rows_unit + r;
+            const int i = ridx / p.G, hq = uh * p.G + (ridx - i * p.G);
+            return (((size_t)ub * p.N + i) * p.Hq + hq) * D;
+        };
+        // Finished unit: O^T (lane = head dim, column = row) is read from TMEM once
+        // the unit's last PV has landed, and the row sums of p are reduced over the
+        // 128 key lanes. A unit this CTA covered whole is normalised and written
+        // out directly; otherwise the CTA stores a partial (unnormalised O, running
+        // maximum, row sum) in its workspace slot for the combine kernel.
+        auto finalize = [&](int jt_last) -> bool {
+            if (!wait_w(&o_full[jt_last & 1], (jt_last >> 1) & 1)) return false;
+            tc_fence_after();
+            float o[CW];
+            tmem_ld_cols<CW>(lane_base + (2 + (lu & 1)) * RPa + col0, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            warp_arrive(&o_free[lu & 1]);
 #pragma unroll
-            for (int c = 0; c < RPh; ++c) {
+            for (int c = 0; c < CW; ++c) {
                 const float v = warp_sum(lsum[c]);
-                if (lane == 0) lred[(wg * 4 + wiw) * RPh + c] = v;
+                if (lane == 0) lred[(wg * 4 + wiw) * CW + c] = v;
+                lsum[c] = 0.f;
             }
             if (!wg_sync()) return false;
+            if (wiw == 0 && lane < CW) {
+                float l = 0.f;
+                for (int w = 0; w < 4; ++w) l += lred[(wg * 4 + w) * CW + lane];
+                lfin[col0 + lane] = l;
+            }
+            if (!wg_sync()) return false;
+            const int Tb = TP[ub + 1] - TP[ub];
+            const int tpre = ups * TP[ub] + (uh * p.RC + urc) * Tb;
+            const int first_cta = tpre / W;
+            const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
+            if (nseg == 1) {
+                if (ell < D) {
+#pragma unroll
+                    for (int c = 0; c < CW; ++c) {
+                        const int r = col0 + c;
+                        if (r < urows) {
+                            const float l = lfin[r];
+                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
+                            p.out[out_row(r) + ell] = *reinterpret_cast<const uint16_t *>(&v);
+                        }
+                    }
+                }
+                return true;
+            }
             float *slot = p.ws_partial + (size_t)(cur_u + blockIdx.x) * slot_floats;
             if (ell < D) {
 #pragma unroll
-                for (int c = 0; c < RPh; ++c)
-                    if (col0 + c < urows) slot[(size_t)(col0 + c) * D + ell] = acc[c];
+                for (int c = 0; c < CW; ++c)
+                    if (col0 + c < urows) slot[(size_t)(col0 + c) * D + ell] = o[c];
             }
-            if (wiw == 0) {
-                for (int c = lane; c < RPh; c += 32) {
-                    const int r = col0 + c;
-                    if (r < urows) {
-                        float l = 0.f;
-                        for (int w = 0; w < 4; ++w) l += lred[(wg * 4 + w) * RPh + c];
-                        slot[(size_t)p.rows_unit * D + r] = mS[last_par * RP + r];
-                        slot[(size_t)p.rows_unit * D + p.rows_unit + r] = l;
-                    }
-                }
+            if (wiw == 0 && lane < CW && col0 + lane < urows) {
+                slot[(size_t)p.rows_unit * D + col0 + lane] = mS[last_par * RP + col0 + lane];
+                slot[(size_t)p.rows_unit * D + p.rows_unit + col0 + lane] = lfin[col0 + lane];
             }
-#pragma unroll
-            for (int c = 0; c < RPh; ++c) { acc[c] = 0.f; lsum[c] = 0.f; }
             return true;
         };
 
@@ -468,10 +525,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
             const bool first = (lt == 0 || ti.j == 0);
             if (first) {
-                if (lt > 0) {
-                    if (!(ok = correction(lt - 1))) break;
-                    if (!(ok = finalize())) break;
-                }
+                if (lt > 0 && !(ok = finalize(lt - 1))) break;
+                ++lu;
                 cur_u = ti.b * ups + ti.hr;
                 ub = ti.b;
                 uh = ti.hr / p.RC;
@@ -484,12 +539,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     if (!(ok = wg_sync())) break;
                 }
             }
-            // ---- softmax of tile lt ----
             const int sb = lt & 1, par = lt & 1;
             if (!(ok = wait_w(&s_full[sb], (lt >> 1) & 1))) break;
             tc_fence_after();
-            float sv[RPh];
-            tmem_ld_cols<RPh>(lane_base + sb * RPa + col0, sv);
+            float sv[CW];
+            tmem_ld_cols<CW>(lane_base + sb * RPa + col0, sv);
             tmem_wait_ld();
             tc_fence_before();
             warp_arrive(&s_empty[sb]);
@@ -503,7 +557,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                 // tile holds keys past ctx_len or new (masked) keys: per-element visibility
                 const int ibase = urc * P.Nc;
 #pragma unroll
-                for (int c = 0; c < RPh; ++c) {
+                for (int c = 0; c < CW; ++c) {
                     bool vis = valid;
                     if (valid && newk >= 0 && col0 + c < urows) {
                         const int i = ibase + rowi[col0 + c];
@@ -512,61 +566,86 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                     if (!vis) sv[c] = -INFINITY;
                 }
             }
+
             // Running maxima are only raised when a score exceeds its column's
             // current maximum by more than 2^RESCALE_LOG2 (after a unit's first
-            // tile this is rare): p = 2^(s*scale - m) then stays below 2^8, and
-            // the tile is folded in with alpha = 1. Otherwise the column maxima
-            // of the tile are reduced over the 128 keys and the state rescaled.
+            // tile this is rare): p = 2^(s*scale - m) then stays below 2^8 and
+            // the tile folds in with alpha = 1. Otherwise the tile's column
+            // maxima are reduced over the 128 keys, the maxima raised, and the
+            // unit's O in TMEM rescaled before this tile's PV adds to it.
             constexpr float RESCALE_LOG2 = 8.f;
             const float sc = p.scale_log2;
-            const float *mo = mS + (par ^ 1) * RP + col0;
+            const float4 *mo4 = reinterpret_cast<const float4 *>(mS + (par ^ 1) * RP + col0);
             bool need = first;
             if (!first) {
 #pragma unroll
-                for (int c = 0; c < RPh; ++c) need |= sv[c] * sc > mo[c] + RESCALE_LOG2;
+                for (int c4 = 0; c4 < CW / 4; ++c4) {
+                    const float4 m4 = mo4[c4];
+                    need |= sv[c4 * 4 + 0] * sc > m4.x + RESCALE_LOG2;
+                    need |= sv[c4 * 4 + 1] * sc > m4.y + RESCALE_LOG2;
+                    need |= sv[c4 * 4 + 2] * sc > m4.z + RESCALE_LOG2;
+                    need |= sv[c4 * 4 + 3] * sc > m4.w + RESCALE_LOG2;
+                }
             }
             const bool wneed = __any_sync(0xffffffffu, need);
-            if (lane == 0) vote[(par * 2 + wg) * 4 + wiw] = wneed;
+            if (lane == 0) vote[(par * NWG + wg) * 4 + wiw] = wneed;
             if (!(ok = wg_sync())) break;
-            const bool rescale = vote[(par * 2 + wg) * 4 + 0] | vote[(par * 2 + wg) * 4 + 1] |
-                                 vote[(par * 2 + wg) * 4 + 2] | vote[(par * 2 + wg) * 4 + 3];
+            const int *vt = vote + (par * NWG + wg) * 4;
+            const bool rescale = (vt[0] | vt[1] | vt[2] | vt[3]) != 0;
             if (rescale) {
-                float *rd = red + ((par * 2 + wg) * 4 + wiw) * RPh;
+                float *rd = red + ((par * NWG + wg) * 4 + wiw) * CW;
 #pragma unroll
-                for (int c = 0; c < RPh; ++c) {
+                for (int c = 0; c < CW; ++c) {
                     float m;
                     asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(m) : "f"(sv[c]));
-                    if (lane == (c & 31)) rd[c] = m;
+                    if (lane == c) rd[c] = m;
                 }
                 if (!(ok = wg_sync())) break;
-                if (wiw == 0) {
-                    for (int c = lane; c < RPh; c += 32) {
-                        const float m_old = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
-                        float rmax = -INFINITY;
-                        for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * 2 + wg) * 4 + w) * RPh + c]);
-                        const float mx = fmaxf(m_old, rmax * sc);
-                        mS[par * RP + col0 + c] = mx;
-                        aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(m_old - mx);
+                if (wiw == 0 && lane < CW) {
+                    const int c = lane;
+                    const float m_old = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
+                    float rmax = -INFINITY;
+                    for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * NWG + wg) * 4 + w) * CW + c]);
+                    const float mx = fmaxf(m_old, rmax * sc);
+                    mS[par * RP + col0 + c] = mx;
+                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(m_old - mx);
+                }
+                if (!(ok = wg_sync())) break;
+                if (!first) {
+                    // scale the unit's O^T columns once the previous tile's PV has landed
+                    if (!(ok = wait_w(&o_full[(lt - 1) & 1], ((lt - 1) >> 1) & 1))) break;
+                    tc_fence_after();
+                    float o[CW];
+                    const uint32_t oaddr = lane_base + (2 + (lu & 1)) * RPa + col0;
+                    tmem_ld_cols<CW>(oaddr, o);
+                    tmem_wait_ld();
+                    const float4 *a4p = reinterpret_cast<const float4 *>(aS + par * RP + col0);
+#pragma unroll
+                    for (int c4 = 0; c4 < CW / 4; ++c4) {
+                        const float4 a4 = a4p[c4];
+                        o[c4 * 4 + 0] *= a4.x;
+                        o[c4 * 4 + 1] *= a4.y;
+                        o[c4 * 4 + 2] *= a4.z;
+                        o[c4 * 4 + 3] *= a4.w;
                     }
+                    tmem_st16(oaddr, o);
+                    tmem_wait_st();
+                    tc_fence_before();
                 }
-                if (!(ok = wg_sync())) break;
-            } else if (wiw == 0) {
-                // keep the maxima; the previous tile's state needs no rescale.
-                // Readers of these slots are past the next tile's first sync.
-                for (int c = lane; c < RPh; c += 32) {
-                    mS[par * RP + col0 + c] = mo[c];
-                    aS[par * RP + col0 + c] = 1.f;
-                }
+            } else if (wiw == 0 && lane < CW) {
+                // keep the maxima: readers of these slots are past the next tile's vote sync
+                mS[par * RP + col0 + lane] = mS[(par ^ 1) * RP + col0 + lane];
+                aS[par * RP + col0 + lane] = 1.f;
             }
             last_par = par;
-            const float *msrc = rescale ? mS + par * RP + col0 : mo;
-            const float *asrc = aS + par * RP + col0;
-            const float4 *ms4 = reinterpret_cast<const float4 *>(msrc);
-            uint32_t packed[RPh / 2];
+            const float4 *ms4 = reinterpret_cast<const float4 *>(rescale ? mS + par * RP + col0
+                                                                         : mS + (par ^ 1) * RP + col0);
+            uint32_t packed[CW / 2];
 #pragma unroll
-            for (int c4 = 0; c4 < RPh / 4; ++c4) {
+            for (int c4 = 0; c4 < CW / 4; ++c4) {
                 const float4 m4 = ms4[c4];
-                const float4 a4 = rescale ? reinterpret_cast<const float4 *>(asrc)[c4] : make_float4(1.f, 1.f, 1.f, 1.f);
+                const float4 a4 = rescale ? reinterpret_cast<const float4 *>(aS + par * RP + col0)[c4]
+                                          : make_float4(1.f, 1.f, 1.f, 1.f);
                 const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, aa[4] = {a4.x, a4.y, a4.z, a4.w};
                 float pp[4];
 #pragma unroll
@@ -585,7 +664,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
             if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
             uint8_t *pbuf = base + L.off_p + pb * L.p_bytes;
 #pragma unroll
-            for (int c8 = 0; c8 < RPh / 8; ++c8) {
+            for (int c8 = 0; c8 < CW / 8; ++c8) {
                 const int cc = col0 + c8 * 8;
                 const int chunk = (cc & 63) >> 3;
                 uint4 *dst = reinterpret_cast<uint4 *>(pbuf + (cc >> 6) * ATOM + (ell >> 3) * 1024 +
@@ -596,43 +675,39 @@ __global__ void __launch_bounds__(TC_THREADS, 1) attn_tc_kernel(const __grid_con
                 // a key past ctx_len: its V row may hold anything (NaN) and P = 0 does not
                 // cancel it, so the row is zeroed once the tile's V has landed
                 if (!(ok = wait_w(&v_full[lt % NV], (lt / NV) & 1))) break;
-            }
-            if (!valid && wg == 0) {
-                uint8_t *vrow = base + (lt % NV) * L.tile_bytes + ell * 128;
-                for (int a = 0; a < nDA; ++a)
-                    for (int q = 0; q < 8; ++q)
-                        reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
+                if (!valid) {
+                    uint8_t *vrow = base + (lt % NV) * L.tile_bytes + ell * 128;
+                    for (int a = 0; a < nDA; ++a)
+                        for (int q = 0; q < 8; ++q)
+                            reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
+                }
             }
             fence_proxy_async_smem();
             warp_arrive(&p_full[pb]);
-            // ---- rescale-and-add the previous tile of the same unit ----
-            if (!first)
-                if (!(ok = correction(lt - 1))) break;
         }
-        if (ok && ntiles > 0) {
-            if (correction(ntiles - 1)) finalize();
-        }
+        if (ok && ntiles > 0) finalize(ntiles - 1);
     }
 
     // ----------------------------- teardown -------------------------------
     tc_fence_before();
     __syncthreads();
-    if (*abort_flag && tid == 0) atomicExch(reinterpret_cast<unsigned int *>(p.ws_plan + p.B + 3), P.epoch);
-    if (warp == 1) {
+    if (*abort_flag && p.status)
+        for (int b = tid; b < p.B; b += NTHREADS) atomicOr(p.status + b, SV_FLAG_TIMEOUT);
+    if (warp == WARP_MMA) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
 }
 
-// ---------------------------------------------------------------------------
-// Combine: merge a unit's partials, normalise, write bf16; one CTA per
-// (row of a unit, unit), one thread per head dimension. The CTA of row 0 of
-// each sequence's first unit also writes that sequence's status flags.
-// ---------------------------------------------------------------------------
 constexpr int COMBINE_MAX_SEGS = 512;  // > num_ctas + 1 on any current GPU
 
-__global__ void attn_combine_kernel(const AttnParams p, uint32_t epoch) {
+// Merge the partials of every unit that was split over several CTAs (a unit one
+// CTA covered whole was written by the attention kernel, and an invalid
+// sequence by its status warp). One CTA per (row of a unit, unit), one thread
+// per head dimension: the segments' (m, l) are loaded in parallel, weighted by
+// 2^(m_k - M), and the partial rows merged.
+__global__ void attn_combine_kernel(const AttnParams p) {
     const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
     const int D = p.D, RU = p.rows_unit;
     const int ups = p.Hkv * p.RC;
@@ -640,71 +715,55 @@ __global__ void attn_combine_kernel(const AttnParams p, uint32_t epoch) {
     const int h = hr / p.RC, rc = hr - h * p.RC;
     const int rows = min(RU, p.R - rc * RU);
     if (r >= rows) return;
-    const int ridx = rc * RU + r;
-    const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const int W = p.ws_plan[0];
     const int *TP = p.ws_plan + 2;
     const int Tb = TP[b + 1] - TP[b];
-    const size_t slot_floats = (size_t)RU * D + 2 * RU;
+    if (Tb == 0) return;
+    const int tpre = ups * TP[b] + hr * Tb;
+    const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
+    if (n == 1) return;
+    const int ridx = rc * RU + r;
+    const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
+    const size_t slot_floats = slot_stride(RU, D);
     __shared__ float sw[COMBINE_MAX_SEGS];
     __shared__ float red_m[4], red_l[4];
+    const float *seg0 = p.ws_partial + (size_t)(u + first) * slot_floats;
+    float m = -INFINITY;
+    for (int k = d; k < n; k += nt) m = fmaxf(m, seg0[(size_t)k * slot_floats + (size_t)RU * D + r]);
+    m = warp_max(m);
+    if ((d & 31) == 0) red_m[d >> 5] = m;
+    __syncthreads();
+    float M = red_m[0];
+    for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_m[w]);
+    float L = 0.f;
+    for (int k = d; k < n; k += nt) {
+        const float *sg = seg0 + (size_t)k * slot_floats;
+        const float mk = sg[(size_t)RU * D + r];
+        const float wk = (mk == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mk - M);
+        sw[k] = wk;
+        L = fmaf(wk, sg[(size_t)RU * D + RU + r], L);
+    }
+    L = warp_sum(L);
+    if ((d & 31) == 0) red_l[d >> 5] = L;
+    __syncthreads();
+    L = 0.f;
+    for (int w = 0; w < (nt + 31) / 32; ++w) L += red_l[w];
     float res = 0.f;
-    if (Tb > 0) {
-        const int tpre = ups * TP[b] + hr * Tb;
-        const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
-        const float *seg0 = p.ws_partial + (size_t)(u + first) * slot_floats;
-        // the segments' (m, l) in parallel, one segment per thread
-        float m = -INFINITY;
-        for (int k = d; k < n; k += nt) m = fmaxf(m, seg0[(size_t)k * slot_floats + (size_t)RU * D + r]);
-        m = warp_max(m);
-        if ((d & 31) == 0) red_m[d >> 5] = m;
-        __syncthreads();
-        float M = red_m[0];
-        for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_m[w]);
-        float L = 0.f;
-        for (int k = d; k < n; k += nt) {
-            const float *sg = seg0 + (size_t)k * slot_floats;
-            const float mk = sg[(size_t)RU * D + r];
-            const float wk = (mk == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mk - M);
-            sw[k] = wk;
-            L = fmaf(wk, sg[(size_t)RU * D + RU + r], L);
-        }
-        L = warp_sum(L);
-        if ((d & 31) == 0) red_l[d >> 5] = L;
-        __syncthreads();
-        L = 0.f;
-        for (int w = 0; w < (nt + 31) / 32; ++w) L += red_l[w];
-        if (L > 0.f) {
-            float acc = 0.f;
+    if (L > 0.f) {
+        float acc = 0.f;
 #pragma unroll 4
-            for (int k = 0; k < n; ++k) acc = fmaf(sw[k], seg0[(size_t)k * slot_floats + (size_t)r * D + d], acc);
-            res = acc / L;
-        }
+        for (int k = 0; k < n; ++k) acc = fmaf(sw[k], seg0[(size_t)k * slot_floats + (size_t)r * D + d], acc);
+        res = acc / L;
     }
     const __nv_bfloat16 o = __float2bfloat16_rn(res);
     p.out[(((size_t)b * p.N + i) * p.Hq + hq) * D + d] = *reinterpret_cast<const uint16_t *>(&o);
-
-    if (p.status && r == 0 && hr == 0) {
-        const int C = p.ctx_lens[b];
-        const bool ctx_ok = C >= p.N && C <= p.max_blocks * PAGE;
-        int bad = 0;
-        if (ctx_ok)
-            for (int jb = d; jb < (C + PAGE - 1) / PAGE; jb += blockDim.x) {
-                const int blk = p.block_table[(size_t)b * p.max_blocks + jb];
-                bad |= (blk < 0 || blk >= p.num_blocks);
-            }
-        bad = __syncthreads_or(bad);
-        if (d == 0) {
-            const bool timed_out = (uint32_t)p.ws_plan[p.B + 3] == epoch;
-            p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0) |
-                          (timed_out ? SV_FLAG_TIMEOUT : 0);
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
+// Workspace: the schedule (tiles per CTA, total, per-sequence tile prefix), then
+// the partial slots.
 static size_t plan_bytes(int B) { return (((size_t)(B + 4) * 4) + 255) & ~(size_t)255; }
 
 void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc) {
@@ -732,7 +791,7 @@ size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_c
     int RU, RC, Nc;
     row_chunks(N, Hq / Hkv, &RU, &RC, &Nc);
     const size_t units = (size_t)B * Hkv * RC;
-    const size_t slot_floats = (size_t)RU * D + 2 * RU;
+    const size_t slot_floats = slot_stride(RU, D);
     return plan_bytes(B) + (units + (size_t)num_ctas) * slot_floats * sizeof(float);
 }
 
@@ -751,16 +810,19 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-static bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D) {
+// Pool map: boxes of 16 keys x 64 dims, 128B-swizzled, for the shared-memory
+// tiles; with whole_page, 16 keys x D dims un-swizzled, for L2 prefetches.
+static bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D,
+                            bool whole_page = false) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)PAGE, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};
     const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)PAGE * D * 2, (cuuint64_t)Hkv * PAGE * D * 2};
-    const cuuint32_t box[4] = {64, PAGE, 1, 1};
+    const cuuint32_t box[4] = {whole_page ? (cuuint32_t)D : 64u, PAGE, 1, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(pool), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, whole_page ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 static bool encode_q_map(CUtensorMap *m, const void *q, int B, int N, int Hq, int D, int G, int Nc) {
@@ -795,7 +857,7 @@ static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
     auto kfn = attn_tc_kernel<D, RP>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kfn<<<P.a.num_ctas, TC_THREADS, smem, stream>>>(P);
+    kfn<<<P.a.num_ctas, tc_threads(RP), smem, stream>>>(P);
     return cudaGetLastError();
 }
 
@@ -832,7 +894,7 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     const int RP = (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3(RU, p.units), p.D, 0, stream>>>(p, P.epoch);
+    attn_combine_kernel<<<dim3(RU, p.units), p.D, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

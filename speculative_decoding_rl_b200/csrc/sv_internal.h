@@ -49,9 +49,8 @@ struct AttnParams {
     const uint64_t *mask;      // [B][N] or null
     uint16_t *out;             // bf16 bits [B][N][Hq][D]
     int32_t *status;           // [B] or null
-    float *ws_partial;         // slots x (rows*D + 2*rows) floats
-    int32_t *ws_plan;          // [0] tiles per CTA, [1] total tiles, [2..2+B] tile prefix per sequence,
-                               // [B+3] epoch of the last call that timed out
+    float *ws_partial;         // partial slots (see slot_stride)
+    int32_t *ws_plan;          // [0] tiles per CTA, [1] total tiles, [2..2+B] tile prefix per sequence
     int B, N, Hq, Hkv, D, G, R, RC, rows_unit, max_blocks, num_blocks;
     int units;                 // B * Hkv * RC
     int num_ctas;
