@@ -117,9 +117,7 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
     p.units = p.B * p.Hkv * p.RC;
     p.num_ctas = ctas;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
-    const size_t plan = sv::attention_plan_bytes(p.B);
-    p.ws_plan = static_cast<int32_t *>(workspace);
-    p.ws_partial = reinterpret_cast<float *>(static_cast<char *>(workspace) + plan);
+    p.ws_partial = static_cast<float *>(workspace);
     cudaError_t e = sv::launch_attention(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(SV_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return SV_OK;

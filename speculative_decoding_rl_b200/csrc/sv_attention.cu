@@ -250,6 +250,11 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
         for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += NTHREADS) q4[e] = make_uint4(0, 0, 0, 0);
     }
+    // Everything above touches only this CTA's shared memory, TMEM and the
+    // kernel parameters, so with a programmatic launch it overlaps the previous
+    // kernel's tail. No input is read, and nothing written, before this wait.
+    griddep_wait();
+    griddep_launch_dependents();  // the combine kernel may now be scheduled
     tile_prefix(p, TP, scratch, CL);  // contains __syncthreads
     fence_proxy_async_smem();
     tc_fence_before();
@@ -260,10 +265,6 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     const int ups = p.Hkv * p.RC;
     const int total = ups * TP[p.B];
     const int W = total > 0 ? (total + p.num_ctas - 1) / p.num_ctas : 1;
-    if (blockIdx.x == 0) {  // the combine kernel's copy of the schedule
-        if (tid == 0) { p.ws_plan[0] = W; p.ws_plan[1] = total; }
-        for (int b = tid; b <= p.B; b += NTHREADS) p.ws_plan[2 + b] = TP[b];
-    }
     const int t_begin = min((int)blockIdx.x * W, total);
     const int t_end = min(t_begin + W, total);
     const int ntiles = t_end - t_begin;
@@ -701,13 +702,30 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
 }
 
 constexpr int COMBINE_MAX_SEGS = 512;  // > num_ctas + 1 on any current GPU
+constexpr int COMBINE_REG_SEGS = 8;    // segments whose partial column is loaded up front
+
+// Block-wide sum / max for blockDim.x <= 128 (at most 4 warps); red holds 4 slots.
+SV_DEV int block_sum_i(int v, int *red) {
+    v = __reduce_add_sync(0xffffffffu, v);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    int t = 0;
+    for (int w = 0; w < (int)(blockDim.x + 31) / 32; ++w) t += red[w];
+    __syncthreads();
+    return t;
+}
 
 // Merge the partials of every unit that was split over several CTAs (a unit one
 // CTA covered whole was written by the attention kernel, and an invalid
 // sequence by its status warp). One CTA per (row of a unit, unit), one thread
-// per head dimension: the segments' (m, l) are loaded in parallel, weighted by
-// 2^(m_k - M), and the partial rows merged.
-__global__ void attn_combine_kernel(const AttnParams p) {
+// per head dimension:
+//   M = max_k m_k,  L = sum_k 2^(m_k - M) l_k,  out = sum_k 2^(m_k - M) O_k / L.
+// Launched as a programmatic dependent of the attention kernel, which lets it
+// launch only after its own wait on earlier work: the schedule is recomputed
+// from ctx_lens (complete by then) before this kernel waits, so once the
+// attention kernel completes one round of loads remains.
+__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+    griddep_launch_dependents();  // the next call's attention kernel may run its prologue
     const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
     const int D = p.D, RU = p.rows_unit;
     const int ups = p.Hkv * p.RC;
@@ -715,56 +733,83 @@ __global__ void attn_combine_kernel(const AttnParams p) {
     const int h = hr / p.RC, rc = hr - h * p.RC;
     const int rows = min(RU, p.R - rc * RU);
     if (r >= rows) return;
-    const int W = p.ws_plan[0];
-    const int *TP = p.ws_plan + 2;
-    const int Tb = TP[b + 1] - TP[b];
+    __shared__ int red_i[4];
+    __shared__ float red_f[4];
+    __shared__ float sw[COMBINE_MAX_SEGS];
+    // the attention kernel's schedule: all tiles, those before sequence b, b's own
+    int tot = 0, before = 0, own = 0;
+    for (int s = d; s < p.B; s += nt) {
+        const int t = seq_tiles(p, s);
+        tot += t;
+        before += s < b ? t : 0;
+        own += s == b ? t : 0;
+    }
+    tot = block_sum_i(tot, red_i);
+    before = block_sum_i(before, red_i);
+    const int Tb = block_sum_i(own, red_i);
     if (Tb == 0) return;
-    const int tpre = ups * TP[b] + hr * Tb;
+    const int total = ups * tot;
+    const int W = (total + p.num_ctas - 1) / p.num_ctas;
+    const int tpre = ups * before + hr * Tb;
     const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
     if (n == 1) return;
     const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const size_t slot_floats = slot_stride(RU, D);
-    __shared__ float sw[COMBINE_MAX_SEGS];
-    __shared__ float red_m[4], red_l[4];
     const float *seg0 = p.ws_partial + (size_t)(u + first) * slot_floats;
-    float m = -INFINITY;
-    for (int k = d; k < n; k += nt) m = fmaxf(m, seg0[(size_t)k * slot_floats + (size_t)RU * D + r]);
+
+    griddep_wait();  // the partials are complete and visible
+    // one round of loads: this thread's column of the first partials, and the
+    // (m, l) of segment d
+    float ov[COMBINE_REG_SEGS];
+#pragma unroll
+    for (int k = 0; k < COMBINE_REG_SEGS; ++k)
+        ov[k] = k < n ? __ldcg(seg0 + (size_t)k * slot_floats + (size_t)r * D + d) : 0.f;
+    float mk = -INFINITY, lk = 0.f;
+    if (d < n) {
+        mk = __ldcg(seg0 + (size_t)d * slot_floats + (size_t)RU * D + r);
+        lk = __ldcg(seg0 + (size_t)d * slot_floats + (size_t)RU * D + RU + r);
+    }
+    float m = mk;
+    for (int k = d + nt; k < n; k += nt) m = fmaxf(m, __ldcg(seg0 + (size_t)k * slot_floats + (size_t)RU * D + r));
     m = warp_max(m);
-    if ((d & 31) == 0) red_m[d >> 5] = m;
+    if ((d & 31) == 0) red_f[d >> 5] = m;
     __syncthreads();
-    float M = red_m[0];
-    for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_m[w]);
+    float M = red_f[0];
+    for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_f[w]);
+    __syncthreads();
+    float lw = 0.f;
+    if (d < n) {
+        const float w = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
+        sw[d] = w;
+        lw = w * lk;
+    }
+    for (int k = d + nt; k < n; k += nt) {
+        const float *sg = seg0 + (size_t)k * slot_floats + (size_t)RU * D;
+        const float mkk = __ldcg(sg + r);
+        const float w = (mkk == -INFINITY) ? 0.f : exp2f(mkk - M);
+        sw[k] = w;
+        lw = fmaf(w, __ldcg(sg + RU + r), lw);
+    }
+    lw = warp_sum(lw);
+    if ((d & 31) == 0) red_f[d >> 5] = lw;
+    __syncthreads();  // also publishes sw
     float L = 0.f;
-    for (int k = d; k < n; k += nt) {
-        const float *sg = seg0 + (size_t)k * slot_floats;
-        const float mk = sg[(size_t)RU * D + r];
-        const float wk = (mk == -INFINITY || M == -INFINITY) ? 0.f : exp2f(mk - M);
-        sw[k] = wk;
-        L = fmaf(wk, sg[(size_t)RU * D + RU + r], L);
-    }
-    L = warp_sum(L);
-    if ((d & 31) == 0) red_l[d >> 5] = L;
-    __syncthreads();
-    L = 0.f;
-    for (int w = 0; w < (nt + 31) / 32; ++w) L += red_l[w];
-    float res = 0.f;
-    if (L > 0.f) {
-        float acc = 0.f;
-#pragma unroll 4
-        for (int k = 0; k < n; ++k) acc = fmaf(sw[k], seg0[(size_t)k * slot_floats + (size_t)r * D + d], acc);
-        res = acc / L;
-    }
-    const __nv_bfloat16 o = __float2bfloat16_rn(res);
+    for (int w = 0; w < (nt + 31) / 32; ++w) L += red_f[w];
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < COMBINE_REG_SEGS; ++k)
+        if (k < n) acc = fmaf(sw[k], ov[k], acc);
+    for (int k = COMBINE_REG_SEGS; k < n; ++k)
+        acc = fmaf(sw[k], __ldcg(seg0 + (size_t)k * slot_floats + (size_t)r * D + d), acc);
+    const __nv_bfloat16 o = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
     p.out[(((size_t)b * p.N + i) * p.Hq + hq) * D + d] = *reinterpret_cast<const uint16_t *>(&o);
 }
 
 // ---------------------------------------------------------------------------
 // Host side.
 // ---------------------------------------------------------------------------
-// Workspace: the schedule (tiles per CTA, total, per-sequence tile prefix), then
-// the partial slots.
-static size_t plan_bytes(int B) { return (((size_t)(B + 4) * 4) + 255) & ~(size_t)255; }
+// Workspace: the partial slots (the combine kernel recomputes the schedule).
 
 void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc) {
     const int R = N * G;
@@ -792,10 +837,8 @@ size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_c
     row_chunks(N, Hq / Hkv, &RU, &RC, &Nc);
     const size_t units = (size_t)B * Hkv * RC;
     const size_t slot_floats = slot_stride(RU, D);
-    return plan_bytes(B) + (units + (size_t)num_ctas) * slot_floats * sizeof(float);
+    return (units + (size_t)num_ctas) * slot_floats * sizeof(float);
 }
-
-size_t attention_plan_bytes(int B) { return plan_bytes(B); }
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -839,6 +882,25 @@ static bool encode_q_map(CUtensorMap *m, const void *q, int B, int N, int Hq, in
 
 constexpr int SMEM_LIMIT = 227 * 1024;
 
+// Launch with programmatic stream serialization: the kernel may start while the
+// previous kernel in the stream finishes; it waits (griddep_wait) before it
+// reads any input or writes anything.
+template <typename... Args>
+static cudaError_t launch_programmatic(void (*kfn)(Args...), dim3 grid, dim3 block, size_t smem,
+                                       cudaStream_t stream, const Args &...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kfn, args...);
+}
+
 template <int D, int RP>
 static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
     // deepest K/V rings and P buffering that fit, in order of preference
@@ -857,8 +919,7 @@ static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
     auto kfn = attn_tc_kernel<D, RP>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kfn<<<P.a.num_ctas, tc_threads(RP), smem, stream>>>(P);
-    return cudaGetLastError();
+    return launch_programmatic(kfn, dim3(P.a.num_ctas), dim3(tc_threads(RP)), smem, stream, P);
 }
 
 template <int D>
@@ -894,8 +955,7 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     const int RP = (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess) return e;
-    attn_combine_kernel<<<dim3(RU, p.units), p.D, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_programmatic(attn_combine_kernel, dim3(RU, p.units), dim3(p.D), 0, stream, p);
 }
 
 }  // namespace sv

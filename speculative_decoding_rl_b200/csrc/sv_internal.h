@@ -50,7 +50,6 @@ struct AttnParams {
     uint16_t *out;             // bf16 bits [B][N][Hq][D]
     int32_t *status;           // [B] or null
     float *ws_partial;         // partial slots (see slot_stride)
-    int32_t *ws_plan;          // [0] tiles per CTA, [1] total tiles, [2..2+B] tile prefix per sequence
     int B, N, Hq, Hkv, D, G, R, RC, rows_unit, max_blocks, num_blocks;
     int units;                 // B * Hkv * RC
     int num_ctas;
@@ -58,7 +57,6 @@ struct AttnParams {
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
-size_t attention_plan_bytes(int B);
 // Row chunks of a unit: rows_unit rows (i, g) per chunk, RC chunks, Nc whole query rows i per chunk.
 void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc);
 int attention_num_ctas();

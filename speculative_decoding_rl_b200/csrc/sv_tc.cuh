@@ -109,6 +109,14 @@ SV_DEV void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Programmatic dependent launch. wait: block until the grids this one depends
+// on have completed and their memory is visible (returns at once for a normal
+// launch). launch_dependents: the grid launched after this one with the
+// programmatic-serialization attribute may start once every CTA of this grid
+// has issued it or exited.
+SV_DEV void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+SV_DEV void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // --------------------------------- TMA --------------------------------------
 SV_DEV void tma_load_4d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0, int c1, int c2, int c3) {
     asm volatile(

@@ -128,3 +128,25 @@ def test_tree_full_size_sampled_rows():
     want = oracle.attention_rows(a, rows)
     sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_attention_close(sel, want, "tree full size, sampled rows")
+
+
+def test_split_units_need_no_workspace_initialisation():
+    # A 40k-token sequence next to a short one: its units are split over dozens
+    # of CTAs and merged by the last to arrive. The workspace starts as random
+    # bytes (arrival counters from no call), then all ones; every call must give
+    # the oracle's result and the same bits.
+    a = W.make_attention_inputs(5, 16, 2, 128, [40000, 300], seed=37)
+    call = AttentionCall(a)
+    g = torch.Generator().manual_seed(5)
+    call.workspace.copy_(torch.randint(0, 256, tuple(call.workspace.shape), dtype=torch.uint8, generator=g))
+    first = call.run().clone()
+    second = call.run().clone()
+    call.workspace.fill_(255)
+    third = call.run().clone()
+    torch.cuda.synchronize()
+    assert (call.status.cpu().numpy() == 0).all()
+    want, flags = oracle.attention(a)
+    assert not flags.any()
+    got = first.float().cpu().numpy().astype(np.float64)
+    assert_attention_close(got, want, "split units, random workspace")
+    assert torch.equal(first, second) and torch.equal(first, third)
