@@ -425,7 +425,7 @@ def run_ours(args, world, rank, local):
             "hbm_gbs_step": step_bytes / (elapsed_max / K) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": recorded_traffic(w.name),
-                         "kernel": "attn_tc_kernel (split context, in-kernel merge)",
+                         "kernel": "sv_verify_attention call: attn_tc_kernel + attn_combine_kernel",
                          "algorithmic_bytes_per_call": alg_bytes, "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * (2 * layers + 1),
             "clocks": clocks, "parity": parity,
