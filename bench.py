@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="qwen7b_longtail")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
+    ap.add_argument("--num-seqs", type=int, default=None, help="active sequences B (qwen32b_sweep)")
+    ap.add_argument("--gamma", type=int, default=None, help="chain drafts per sequence (qwen32b_sweep)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
@@ -213,10 +215,26 @@ def oracle_sample(w: W.Workload, a0, acc, layers: int, budget_s: float, seed: in
 # arms
 # ---------------------------------------------------------------------------
 
+def make_workload(args):
+    over = {}
+    if args.num_seqs is not None or args.gamma is not None:
+        if args.workload != "qwen32b_sweep":
+            raise SystemExit("--num-seqs / --gamma apply to the qwen32b_sweep workload")
+        if args.num_seqs is not None:
+            over["num_seqs"] = args.num_seqs
+        if args.gamma is not None:
+            over["gamma"] = args.gamma
+    return W.workload(args.workload, **over)
+
+
+# distinct KV pools are kept within this many bytes; layers beyond cycle through
+# them (each pool is then far larger than L2, so no layer finds another's pages cached)
+POOL_BUDGET_BYTES = 48 << 30
+
 def run_reference(args, world, rank):
     if rank != 0:
         return
-    w = W.workload(args.workload)
+    w = make_workload(args)
     layers = args.layers or w.num_layers
     a0 = W.build_attention(w)
     acc = W.build_accept(w)
@@ -243,24 +261,30 @@ def run_ours(args, world, rank, local):
     from speculative_decoding_rl_b200.session import AcceptCall, AttentionCall
 
     dev = torch.device("cuda", local)
-    w = W.workload(args.workload)
+    w = make_workload(args)
     layers = args.layers or w.num_layers
     a0 = W.build_attention(w)
     acc_in = W.build_accept(w)
     B, N, Hq, D = a0.num_seqs, a0.num_q_rows, a0.num_q_heads, a0.head_dim
 
     # Layer 0 from the seeded CPU generator; layers 1.. get their own pools and
-    # queries drawn on the device (same sequences and page tables).
+    # queries drawn on the device (same sequences and page tables). Distinct pools
+    # are capped by POOL_BUDGET_BYTES; past that, layers reuse pools cyclically.
     calls = [AttentionCall(a0, device=str(dev))]
     g = torch.Generator(device=dev)
     g.manual_seed(1234 + rank)
-    for _ in range(1, layers):
+    pool_bytes = 2 * a0.k_pool.numel() * 2
+    n_pools = max(1, min(layers, POOL_BUDGET_BYTES // max(1, pool_bytes)))
+    for li in range(1, layers):
         c = AttentionCall.__new__(AttentionCall)
         c.inputs = a0
         c.desc = calls[0].desc
         c.block_table, c.ctx_lens, c.mask = calls[0].block_table, calls[0].ctx_lens, calls[0].mask
-        c.k_pool = torch.randn(a0.k_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
-        c.v_pool = torch.randn(a0.v_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
+        if li < n_pools:
+            c.k_pool = torch.randn(a0.k_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
+            c.v_pool = torch.randn(a0.v_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
+        else:
+            c.k_pool, c.v_pool = calls[li % n_pools].k_pool, calls[li % n_pools].v_pool
         c.q = torch.randn(a0.q.shape, generator=g, device=dev, dtype=torch.bfloat16)
         c.out = torch.empty_like(c.q)
         c.status = None
@@ -418,7 +442,8 @@ def run_ours(args, world, rank, local):
                        "q_heads": Hq, "kv_heads": a0.num_kv_heads, "head_dim": D,
                        "ctx_tokens_total": int(a0.ctx_lens.sum()), "vocab": acc_in.vocab,
                        "temperature": acc_in.temperature,
-                       "l2": "inputs larger than L2 (every layer has its own KV pool)",
+                       "l2": ("inputs larger than L2 (every layer has its own KV pool)" if n_pools == layers else
+                              f"inputs larger than L2 ({n_pools} KV pools of {pool_bytes / 1e9:.1f} GB cycled over {layers} layers)"),
                        "parallelism": f"replicas x{world}"},
             "accepted_tok_s": tok_s,
             "t_attn_call_ms": 1e3 * t_attn, "t_accept_call_ms": 1e3 * t_acc,

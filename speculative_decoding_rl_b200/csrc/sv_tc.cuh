@@ -139,6 +139,14 @@ SV_DEV void tma_prefetch_l2_4d(const CUtensorMap *map, int c0, int c1, int c2, i
                  "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
+// Contiguous global -> shared copy on the TMA unit (no tensor map): both
+// addresses 16-byte aligned, bytes a multiple of 16; completion is counted on
+// `bar` as transaction bytes. The destination is this CTA's shared memory.
+SV_DEV void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
 SV_DEV void tma_prefetch_desc(const CUtensorMap *map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
