@@ -136,7 +136,7 @@ constexpr uint32_t ATOM = 16384;  // 128 rows x 128 bytes, one 128B-swizzle colu
 
 struct TcLayout {
     uint32_t tile_bytes, off_k, off_q, q_bytes, off_p, p_bytes, off_bar, off_tp, off_cl, off_red, off_ms, off_as,
-        off_lred, off_rowi, off_umask, off_vote, off_fin, off_misc, total;
+        off_lred, off_rowi, off_umask, off_vote, off_fin, off_mfin, off_misc, total;
 };
 
 // V ring first (slots 0..NV-1), then the K ring: a V slot plus 16 KB is always
@@ -164,7 +164,8 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int
     L.off_umask = (L.off_rowi + 4u * RP + 15u) & ~15u;        // [RP] row r -> r / G
     L.off_vote = L.off_umask + 8u * NWG * 64;                 // [wg][64] mask words of the unit
     L.off_fin = L.off_vote + 4u * 2 * NWG * WARPS_PER_WG;     // [par][wg][warp] rescale votes
-    L.off_misc = L.off_fin + 4u * RP;                         // [RP] row sums of a finished unit
+    L.off_mfin = L.off_fin + 4u * RP;                         // [RP] row sums of a finished unit
+    L.off_misc = L.off_mfin + 4u * RP;                        // [RP] row maxima of a finished unit
     L.total = L.off_misc + 16u + 4u * 32;
     return L;
 }
@@ -216,6 +217,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     uint64_t *umask = reinterpret_cast<uint64_t *>(base + L.off_umask);
     int *vote = reinterpret_cast<int *>(base + L.off_vote);
     float *lfin = reinterpret_cast<float *>(base + L.off_fin);  // [RP] row sums of the finished unit
+    float *mfin = reinterpret_cast<float *>(base + L.off_mfin); // [RP] its row maxima
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
     int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // one int per warp (<= 28), used once
@@ -459,25 +461,17 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             wg_phase ^= 1;
             return r;
         };
-        // output row r of the current unit -> element offset of (b, i, hq, 0) in out
-        auto out_row = [&](int r) -> size_t {
-            const int ridx = urc * p.rows_unit + r;
-            const int i = ridx / p.G, hq = uh * p.G + (ridx - i * p.G);
-            return (((size_t)ub * p.N + i) * p.Hq + hq) * D;
-        };
-        // Finished unit: O^T (lane = head dim, column = row) is read from TMEM once
-        // the unit's last PV has landed, and the row sums of p are reduced over the
-        // 128 key lanes. A unit this CTA covered whole is normalised and written
-        // out directly; otherwise the CTA stores a partial (unnormalised O, running
-        // maximum, row sum) in its workspace slot for the combine kernel.
-        auto finalize = [&](int jt_last) -> bool {
-            if (!wait_w(&o_full[jt_last & 1], (jt_last >> 1) & 1)) return false;
-            tc_fence_after();
-            float o[CW];
-            tmem_ld_cols<CW>(lane_base + (2 + (lu & 1)) * RPa + col0, o);
-            tmem_wait_ld();
-            tc_fence_before();
-            warp_arrive(&o_free[lu & 1]);
+        // A unit ends in two steps. close_unit, at the boundary: the row sums of
+        // p are reduced over the 128 key lanes and kept with the row maxima; no
+        // wait on the tensor core. finish_unit, once the next unit's first tile
+        // is through softmax (its last PV has landed by then, or nearly): O^T
+        // (lane = head dim, column = row) is read from the unit's TMEM buffer,
+        // which is then released. A unit this CTA covered whole is normalised
+        // and written out; otherwise the CTA stores a partial (unnormalised O,
+        // running maximum, row sum) in its workspace slot for the combine kernel.
+        bool pending = false;
+        int pend_u = 0, pend_ob = 0, pend_jt = 0;
+        auto close_unit = [&](int jt_last) -> bool {
 #pragma unroll
             for (int c = 0; c < CW; ++c) {
                 const float v = warp_sum(lsum[c]);
@@ -489,10 +483,29 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 float l = 0.f;
                 for (int w = 0; w < 4; ++w) l += lred[(wg * 4 + w) * CW + lane];
                 lfin[col0 + lane] = l;
+                mfin[col0 + lane] = mS[last_par * RP + col0 + lane];
             }
             if (!wg_sync()) return false;
-            const int Tb = TP[ub + 1] - TP[ub];
-            const int tpre = ups * TP[ub] + (uh * p.RC + urc) * Tb;
+            pending = true;
+            pend_u = cur_u;
+            pend_ob = lu & 1;
+            pend_jt = jt_last;
+            return true;
+        };
+        auto finish_unit = [&]() -> bool {
+            pending = false;
+            if (!wait_w(&o_full[pend_jt & 1], (pend_jt >> 1) & 1)) return false;
+            tc_fence_after();
+            float o[CW];
+            tmem_ld_cols<CW>(lane_base + (2 + pend_ob) * RPa + col0, o);
+            tmem_wait_ld();
+            tc_fence_before();
+            warp_arrive(&o_free[pend_ob]);
+            const int fb = pend_u / ups, fhr = pend_u - fb * ups;
+            const int fh = fhr / p.RC, frc = fhr - fh * p.RC;
+            const int frows = min(p.rows_unit, p.R - frc * p.rows_unit);
+            const int Tb = TP[fb + 1] - TP[fb];
+            const int tpre = ups * TP[fb] + fhr * Tb;
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
             if (nseg == 1) {
@@ -500,33 +513,41 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
 #pragma unroll
                     for (int c = 0; c < CW; ++c) {
                         const int r = col0 + c;
-                        if (r < urows) {
+                        if (r < frows) {
                             const float l = lfin[r];
                             const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
-                            p.out[out_row(r) + ell] = *reinterpret_cast<const uint16_t *>(&v);
+                            const int ridx = frc * p.rows_unit + r;
+                            const int i = ridx / p.G, hq = fh * p.G + (ridx - i * p.G);
+                            p.out[(((size_t)fb * p.N + i) * p.Hq + hq) * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
                         }
                     }
                 }
                 return true;
             }
-            float *slot = p.ws_partial + (size_t)(cur_u + blockIdx.x) * slot_floats;
+            float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
             if (ell < D) {
 #pragma unroll
                 for (int c = 0; c < CW; ++c)
-                    if (col0 + c < urows) slot[(size_t)(col0 + c) * D + ell] = o[c];
+                    if (col0 + c < frows) slot[(size_t)(col0 + c) * D + ell] = o[c];
             }
-            if (wiw == 0 && lane < CW && col0 + lane < urows) {
-                slot[(size_t)p.rows_unit * D + col0 + lane] = mS[last_par * RP + col0 + lane];
+            if (wiw == 0 && lane < CW && col0 + lane < frows) {
+                slot[(size_t)p.rows_unit * D + col0 + lane] = mfin[col0 + lane];
                 slot[(size_t)p.rows_unit * D + p.rows_unit + col0 + lane] = lfin[col0 + lane];
             }
             return true;
         };
 
-        for (int lt = 0; lt < ntiles && ok; ++lt) {
-            const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
-            const bool first = (lt == 0 || ti.j == 0);
+        // one pass past the last tile closes and finishes the CTA's last unit
+        for (int lt = 0; lt <= ntiles && ok; ++lt) {
+            const bool end = lt == ntiles;
+            const TileInfo ti = end ? TileInfo{0, 0, 0, 1} : decode_tile(TP, p.B, ups, t_begin + lt);
+            const bool first = (lt == 0 || ti.j == 0 || end);
             if (first) {
-                if (lt > 0 && !(ok = finalize(lt - 1))) break;
+                if (lt > 0 && !(ok = close_unit(lt - 1))) break;
+                if (end) {
+                    if (pending) ok = finish_unit();
+                    break;
+                }
                 ++lu;
                 cur_u = ti.b * ups + ti.hr;
                 ub = ti.b;
@@ -685,8 +706,9 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             }
             fence_proxy_async_smem();
             warp_arrive(&p_full[pb]);
+            // the previous unit's last PV was issued before this tile's
+            if (pending && !(ok = finish_unit())) break;
         }
-        if (ok && ntiles > 0) finalize(ntiles - 1);
     }
 
     // ----------------------------- teardown -------------------------------
