@@ -52,11 +52,17 @@ namespace sv {
 using namespace tc;
 
 // Softmax warpgroups: 4 warps each (one TMEM lane quadrant per warp), each
-// owning CW consecutive row columns; a unit's padded row count RP = CW * NWG.
-constexpr int CW = 16;
+// owning tc_cw(RP) consecutive row columns; RP = tc_cw(RP) * NWG. 96-row units
+// take 32 columns per warpgroup: half the warps, each with twice the registers
+// (no spills) and its fixed per-tile costs paid half as often.
+__host__ __device__ constexpr int tc_cw(int RP) { return RP == 96 ? 32 : 16; }
 constexpr int WARPS_PER_WG = 4;
-__host__ __device__ constexpr int tc_nwg(int RP) { return RP / CW; }
+__host__ __device__ constexpr int tc_nwg(int RP) { return RP / tc_cw(RP); }
 __host__ __device__ constexpr int tc_threads(int RP) { return 32 * (WARPS_PER_WG * tc_nwg(RP) + 4); }
+// Running column maximum of a column that has seen no visible key: finite, so
+// that s*scale - M_NONE is +huge for a visible score (it votes for a raise) and
+// -inf for a masked one (p = 0), with no special case in the exponentials.
+constexpr float M_NONE = -3.402823466e38f;
 constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
 
 // ---------------------------------------------------------------------------
@@ -129,6 +135,20 @@ SV_DEV TileInfo decode_tile(const int *TP, int B, int ups, int t) {
     return ti;
 }
 
+// The tile after ti in the end-to-end order (j, then head/row chunk, then
+// sequence; sequences without tiles are skipped). Callers stop at their range's
+// end, so running past the last sequence only has to be harmless.
+SV_DEV void next_tile(TileInfo &ti, const int *TP, int B, int ups) {
+    if (++ti.j < ti.Tb) return;
+    ti.j = 0;
+    if (++ti.hr < ups) return;
+    ti.hr = 0;
+    do {
+        ++ti.b;
+        ti.Tb = ti.b < B ? TP[ti.b + 1] - TP[ti.b] : 1;
+    } while (ti.b < B && ti.Tb == 0);
+}
+
 // ---------------------------------------------------------------------------
 // Shared-memory plan of the tcgen05 kernel (host and device agree).
 // ---------------------------------------------------------------------------
@@ -141,7 +161,7 @@ struct TcLayout {
 
 // V ring first (slots 0..NV-1), then the K ring: a V slot plus 16 KB is always
 // inside the allocation (the D = 64 PV product reads one unused atom there).
-__host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int NP, int B) {
+__host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int NP, int NQ, int B) {
     TcLayout L;
     const int nDA = D / 64;
     const int NWG = tc_nwg(RP);
@@ -149,7 +169,7 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int
     L.off_k = NV * L.tile_bytes;
     L.off_q = L.off_k + NK * L.tile_bytes;
     L.q_bytes = (uint32_t)nDA * RP * 128u;
-    L.off_p = L.off_q + 2u * L.q_bytes;
+    L.off_p = L.off_q + (uint32_t)NQ * L.q_bytes;
     L.p_bytes = (uint32_t)((RP + 63) / 64) * ATOM;
     L.off_bar = L.off_p + NP * L.p_bytes;
     const int nbar = 2 * NK + 2 * NV + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ +
@@ -157,6 +177,7 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int
     L.off_tp = L.off_bar + 8u * nbar;
     L.off_cl = L.off_tp + 4u * (B + 1);
     L.off_red = (L.off_cl + 4u * B + 15u) & ~15u;
+    const int CW = tc_cw(RP);
     L.off_ms = L.off_red + 4u * 2 * NWG * WARPS_PER_WG * CW;  // [par][wg][warp][CW] tile column maxima
     L.off_as = L.off_ms + 4u * 2 * RP;                        // [par][RP] running maxima
     L.off_lred = L.off_as + 4u * 2 * RP;                      // [par][RP] rescale factors
@@ -175,7 +196,7 @@ struct TcParams {
     CUtensorMap tm_v;
     CUtensorMap tm_q;
     AttnParams a;
-    int NK, NV, NP, Nc;
+    int NK, NV, NP, NQ, Nc;  // K / V / P slots, query buffers (1 or 2), query rows per chunk
     uint32_t epoch;
 };
 
@@ -186,17 +207,21 @@ template <int D, int RP>
 __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid_constant__ TcParams P) {
     constexpr int nDA = D / 64;
     constexpr int NWG = tc_nwg(RP);
+    constexpr int CW = tc_cw(RP);
     constexpr int MATH_WARPS = WARPS_PER_WG * NWG;
     constexpr int NTHREADS = tc_threads(RP);
     constexpr int RPa = (RP + 31) / 32 * 32;  // TMEM columns per S / O buffer
     constexpr int WARP_K = MATH_WARPS, WARP_MMA = MATH_WARPS + 1, WARP_V = MATH_WARPS + 2,
                   WARP_ST = MATH_WARPS + 3;
     const AttnParams &p = P.a;
-    const int NK = P.NK, NV = P.NV, NP = P.NP;
+    const int NK = P.NK, NV = P.NV, NP = P.NP, NQ = P.NQ;
+    // query buffer of the u-th unit and the phase of its barriers
+    auto qbuf = [NQ](int u) { return NQ == 1 ? 0 : (u & 1); };
+    auto qphase = [NQ](int u) -> uint32_t { return NQ == 1 ? (u & 1) : ((u >> 1) & 1); };
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const TcLayout L = tc_layout(D, RP, NK, NV, NP, p.B);
+    const TcLayout L = tc_layout(D, RP, NK, NV, NP, NQ, p.B);
     uint64_t *bar = reinterpret_cast<uint64_t *>(base + L.off_bar);
     uint64_t *k_full = bar, *k_empty = bar + NK;
     uint64_t *v_full = bar + 2 * NK, *v_empty = v_full + NV;
@@ -250,7 +275,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     for (int r = tid; r < RP; r += NTHREADS) rowi[r] = r / p.G;
     {  // zero both query buffers: rows past a unit's real rows stay zero
         uint4 *q4 = reinterpret_cast<uint4 *>(base + L.off_q);
-        for (uint32_t e = tid; e < 2u * L.q_bytes / 16u; e += NTHREADS) q4[e] = make_uint4(0, 0, 0, 0);
+        for (uint32_t e = tid; e < (uint32_t)NQ * L.q_bytes / 16u; e += NTHREADS) q4[e] = make_uint4(0, 0, 0, 0);
     }
     // Everything above touches only this CTA's shared memory, TMEM and the
     // kernel parameters, so with a programmatic launch it overlaps the previous
@@ -282,8 +307,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             uint8_t *ring = base + (is_k ? L.off_k : 0u);
             const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
             int lu = -1, issued_tiles = 0;
-            for (int lt = 0; lt < ntiles; ++lt) {
-                const TileInfo ti = decode_tile(TP, p.B, ups, t_begin + lt);
+            TileInfo ti = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+            for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
                 const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
                 // gather the tile's page ids first (independent loads), then wait for the slot
                 const int C = CL[ti.b];
@@ -295,8 +320,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 }
                 if (is_k && (lt == 0 || ti.j == 0)) {
                     ++lu;
-                    const int qb = lu & 1;
-                    if (!mbar_wait(&q_empty[qb], ((lu >> 1) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                    const int qb = qbuf(lu);
+                    if (!mbar_wait(&q_empty[qb], qphase(lu) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
                     mbar_arrive_expect_tx(&q_full[qb], q_box_bytes * nDA);
                     uint8_t *qdst = base + L.off_q + qb * L.q_bytes;
                     for (int a = 0; a < nDA; ++a)
@@ -322,8 +347,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 for (int lt = max(0, issued_tiles - NR); lt < issued_tiles; ++lt)
                     mbar_wait_time(&full[lt % NR], (lt / NR) & 1, WAIT_LIMIT_NS);
                 if (is_k)
-                    for (int u = max(0, lu - 1); u <= lu; ++u)
-                        mbar_wait_time(&q_full[u & 1], (u >> 1) & 1, WAIT_LIMIT_NS);
+                    for (int u = max(0, lu - NQ + 1); u <= lu; ++u)
+                        mbar_wait_time(&q_full[qbuf(u)], qphase(u), WAIT_LIMIT_NS);
             }
         }
     } else if (warp == WARP_ST) {
@@ -368,9 +393,9 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 if (nq < ntiles) {
                     const bool newu = (nq == 0 || tq.j == 0);
                     const int lu_n = newu ? lu + 1 : lu;
-                    const int qb_n = lu_n & 1;
+                    const int qb_n = qbuf(lu_n);
                     const int s = nq % NK, sb = nq & 1;
-                    if ((!newu || mbar_test(&q_full[qb_n], (lu_n >> 1) & 1)) &&
+                    if ((!newu || mbar_test(&q_full[qb_n], qphase(lu_n))) &&
                         mbar_test(&k_full[s], (nq / NK) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
                         lu = lu_n;
                         qb = qb_n;
@@ -387,7 +412,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         mma_commit(&k_empty[s]);
                         if (nq == ntiles - 1 || tq.j == tq.Tb - 1) mma_commit(&q_empty[qb]);
                         ++nq;
-                        if (nq < ntiles) tq = decode_tile(TP, p.B, ups, t_begin + nq);
+                        if (nq < ntiles) next_tile(tq, TP, p.B, ups);
                         progressed = true;
                     }
                 }
@@ -411,7 +436,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[s]);
                         ++np;
-                        if (np < ntiles) tp = decode_tile(TP, p.B, ups, t_begin + np);
+                        if (np < ntiles) next_tile(tp, TP, p.B, ups);
                         progressed = true;
                     }
                 }
@@ -496,11 +521,6 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             pending = false;
             if (!wait_w(&o_full[pend_jt & 1], (pend_jt >> 1) & 1)) return false;
             tc_fence_after();
-            float o[CW];
-            tmem_ld_cols<CW>(lane_base + (2 + pend_ob) * RPa + col0, o);
-            tmem_wait_ld();
-            tc_fence_before();
-            warp_arrive(&o_free[pend_ob]);
             const int fb = pend_u / ups, fhr = pend_u - fb * ups;
             const int fh = fhr / p.RC, frc = fhr - fh * p.RC;
             const int frows = min(p.rows_unit, p.R - frc * p.rows_unit);
@@ -508,11 +528,18 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const int tpre = ups * TP[fb] + fhr * Tb;
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
-            if (nseg == 1) {
-                if (ell < D) {
+            float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
+            // O^T in chunks of 16 columns (few live registers)
+#pragma unroll 1
+            for (int c0 = 0; c0 < CW; c0 += 16) {
+                float o[16];
+                tmem_ld16(lane_base + (2 + pend_ob) * RPa + col0 + c0, o);
+                tmem_wait_ld();
+                if (ell >= D) continue;
+                if (nseg == 1) {
 #pragma unroll
-                    for (int c = 0; c < CW; ++c) {
-                        const int r = col0 + c;
+                    for (int c = 0; c < 16; ++c) {
+                        const int r = col0 + c0 + c;
                         if (r < frows) {
                             const float l = lfin[r];
                             const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
@@ -521,16 +548,15 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                             p.out[(((size_t)fb * p.N + i) * p.Hq + hq) * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
                         }
                     }
-                }
-                return true;
-            }
-            float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
-            if (ell < D) {
+                } else {
 #pragma unroll
-                for (int c = 0; c < CW; ++c)
-                    if (col0 + c < frows) slot[(size_t)(col0 + c) * D + ell] = o[c];
+                    for (int c = 0; c < 16; ++c)
+                        if (col0 + c0 + c < frows) slot[(size_t)(col0 + c0 + c) * D + ell] = o[c];
+                }
             }
-            if (wiw == 0 && lane < CW && col0 + lane < frows) {
+            tc_fence_before();
+            warp_arrive(&o_free[pend_ob]);
+            if (nseg > 1 && wiw == 0 && lane < CW && col0 + lane < frows) {
                 slot[(size_t)p.rows_unit * D + col0 + lane] = mfin[col0 + lane];
                 slot[(size_t)p.rows_unit * D + p.rows_unit + col0 + lane] = lfin[col0 + lane];
             }
@@ -538,9 +564,11 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         };
 
         // one pass past the last tile closes and finishes the CTA's last unit
+        TileInfo tnext = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
         for (int lt = 0; lt <= ntiles && ok; ++lt) {
             const bool end = lt == ntiles;
-            const TileInfo ti = end ? TileInfo{0, 0, 0, 1} : decode_tile(TP, p.B, ups, t_begin + lt);
+            const TileInfo ti = end ? TileInfo{0, 0, 0, 1} : tnext;
+            if (!end) next_tile(tnext, TP, p.B, ups);
             const bool first = (lt == 0 || ti.j == 0 || end);
             if (first) {
                 if (lt > 0 && !(ok = close_unit(lt - 1))) break;
@@ -595,6 +623,10 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             // the tile folds in with alpha = 1. Otherwise the tile's column
             // maxima are reduced over the 128 keys, the maxima raised, and the
             // unit's O in TMEM rescaled before this tile's PV adds to it.
+            // The exponent s*scale - m against the current maxima decides the vote
+            // and (when nothing is raised) feeds the exponentials. A column with no
+            // visible key yet holds M_NONE: its first visible score votes for a
+            // raise, and masked scores (-inf) give 2^-inf = 0.
             constexpr float RESCALE_LOG2 = 8.f;
             const float sc = p.scale_log2;
             const float4 *mo4 = reinterpret_cast<const float4 *>(mS + (par ^ 1) * RP + col0);
@@ -603,10 +635,10 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
 #pragma unroll
                 for (int c4 = 0; c4 < CW / 4; ++c4) {
                     const float4 m4 = mo4[c4];
-                    need |= sv[c4 * 4 + 0] * sc > m4.x + RESCALE_LOG2;
-                    need |= sv[c4 * 4 + 1] * sc > m4.y + RESCALE_LOG2;
-                    need |= sv[c4 * 4 + 2] * sc > m4.z + RESCALE_LOG2;
-                    need |= sv[c4 * 4 + 3] * sc > m4.w + RESCALE_LOG2;
+                    need |= fmaf(sv[c4 * 4 + 0], sc, -m4.x) > RESCALE_LOG2;
+                    need |= fmaf(sv[c4 * 4 + 1], sc, -m4.y) > RESCALE_LOG2;
+                    need |= fmaf(sv[c4 * 4 + 2], sc, -m4.z) > RESCALE_LOG2;
+                    need |= fmaf(sv[c4 * 4 + 3], sc, -m4.w) > RESCALE_LOG2;
                 }
             }
             const bool wneed = __any_sync(0xffffffffu, need);
@@ -625,32 +657,47 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 if (!(ok = wg_sync())) break;
                 if (wiw == 0 && lane < CW) {
                     const int c = lane;
-                    const float m_old = first ? -INFINITY : mS[(par ^ 1) * RP + col0 + c];
+                    const float m_old = first ? M_NONE : mS[(par ^ 1) * RP + col0 + c];
                     float rmax = -INFINITY;
                     for (int w = 0; w < 4; ++w) rmax = fmaxf(rmax, red[((par * NWG + wg) * 4 + w) * CW + c]);
-                    const float mx = fmaxf(m_old, rmax * sc);
+                    const float mx = fmaxf(m_old, rmax * sc);  // stays M_NONE while nothing is visible
                     mS[par * RP + col0 + c] = mx;
-                    aS[par * RP + col0 + c] = (mx == -INFINITY) ? 1.f : ex2_approx(m_old - mx);
+                    aS[par * RP + col0 + c] = ex2_approx(m_old - mx);  // M_NONE - finite underflows to 0
                 }
                 if (!(ok = wg_sync())) break;
+                {
+                    // the running row sums follow the raised maxima
+                    const float4 *an4 = reinterpret_cast<const float4 *>(aS + par * RP + col0);
+#pragma unroll
+                    for (int c4 = 0; c4 < CW / 4; ++c4) {
+                        const float4 a4 = an4[c4];
+                        lsum[c4 * 4 + 0] *= a4.x;
+                        lsum[c4 * 4 + 1] *= a4.y;
+                        lsum[c4 * 4 + 2] *= a4.z;
+                        lsum[c4 * 4 + 3] *= a4.w;
+                    }
+                }
                 if (!first) {
                     // scale the unit's O^T columns once the previous tile's PV has landed
                     if (!(ok = wait_w(&o_full[(lt - 1) & 1], ((lt - 1) >> 1) & 1))) break;
                     tc_fence_after();
-                    float o[CW];
-                    const uint32_t oaddr = lane_base + (2 + (lu & 1)) * RPa + col0;
-                    tmem_ld_cols<CW>(oaddr, o);
-                    tmem_wait_ld();
-                    const float4 *a4p = reinterpret_cast<const float4 *>(aS + par * RP + col0);
+#pragma unroll 1
+                    for (int c0 = 0; c0 < CW; c0 += 16) {  // chunks of 16 columns
+                        float o[16];
+                        const uint32_t oaddr = lane_base + (2 + (lu & 1)) * RPa + col0 + c0;
+                        tmem_ld16(oaddr, o);
+                        tmem_wait_ld();
+                        const float4 *a4p = reinterpret_cast<const float4 *>(aS + par * RP + col0 + c0);
 #pragma unroll
-                    for (int c4 = 0; c4 < CW / 4; ++c4) {
-                        const float4 a4 = a4p[c4];
-                        o[c4 * 4 + 0] *= a4.x;
-                        o[c4 * 4 + 1] *= a4.y;
-                        o[c4 * 4 + 2] *= a4.z;
-                        o[c4 * 4 + 3] *= a4.w;
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const float4 a4 = a4p[c4];
+                            o[c4 * 4 + 0] *= a4.x;
+                            o[c4 * 4 + 1] *= a4.y;
+                            o[c4 * 4 + 2] *= a4.z;
+                            o[c4 * 4 + 3] *= a4.w;
+                        }
+                        tmem_st16(oaddr, o);
                     }
-                    tmem_st16(oaddr, o);
                     tmem_wait_st();
                     tc_fence_before();
                 }
@@ -660,22 +707,18 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 aS[par * RP + col0 + lane] = 1.f;
             }
             last_par = par;
-            const float4 *ms4 = reinterpret_cast<const float4 *>(rescale ? mS + par * RP + col0
-                                                                         : mS + (par ^ 1) * RP + col0);
+            const float4 *ms4 = reinterpret_cast<const float4 *>(mS + (rescale ? par : par ^ 1) * RP + col0);
             uint32_t packed[CW / 2];
 #pragma unroll
             for (int c4 = 0; c4 < CW / 4; ++c4) {
                 const float4 m4 = ms4[c4];
-                const float4 a4 = rescale ? reinterpret_cast<const float4 *>(aS + par * RP + col0)[c4]
-                                          : make_float4(1.f, 1.f, 1.f, 1.f);
-                const float mm[4] = {m4.x, m4.y, m4.z, m4.w}, aa[4] = {a4.x, a4.y, a4.z, a4.w};
+                const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
                 float pp[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int c = c4 * 4 + k;
-                    // p = 2^(s*scale - m); a column with no visible key yet (m = -inf) gives 0
-                    pp[k] = mm[k] == -INFINITY ? 0.f : ex2_approx(fmaf(sv[c], sc, -mm[k]));
-                    lsum[c] = fmaf(lsum[c], aa[k], pp[k]);
+                    pp[k] = ex2_approx(fmaf(sv[c], sc, -mm[k]));  // p = 2^(s*scale - m)
+                    lsum[c] += pp[k];
                 }
                 __nv_bfloat162 h0 = __floats2bfloat162_rn(pp[0], pp[1]);
                 __nv_bfloat162 h1 = __floats2bfloat162_rn(pp[2], pp[3]);
@@ -925,18 +968,23 @@ static cudaError_t launch_programmatic(void (*kfn)(Args...), dim3 grid, dim3 blo
 
 template <int D, int RP>
 static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
-    // deepest K/V rings and P buffering that fit, in order of preference
-    static const int choices[][3] = {{3, 4, 2}, {2, 4, 2}, {2, 3, 2}, {2, 3, 1}, {2, 2, 2}, {2, 2, 1}};
+    // deepest K/V rings, P and query buffering that fit, in order of preference
+    // (K, V, P, Q); a single query buffer stalls a unit's first product on its
+    // query load, which costs less than a shallower ring when units are long
+    static const int choices[][4] = {{3, 4, 2, 2}, {2, 4, 2, 2}, {2, 3, 2, 2}, {2, 3, 1, 2}, {2, 2, 2, 2},
+                                     {2, 2, 1, 2}, {2, 2, 1, 1}};
+    constexpr int nchoices = sizeof(choices) / sizeof(choices[0]);
     TcLayout L;
     int k = 0;
-    for (; k < 6; ++k) {
-        L = tc_layout(D, RP, choices[k][0], choices[k][1], choices[k][2], P.a.B);
+    for (; k < nchoices; ++k) {
+        L = tc_layout(D, RP, choices[k][0], choices[k][1], choices[k][2], choices[k][3], P.a.B);
         if (L.total + 1024 <= (uint32_t)SMEM_LIMIT) break;
     }
-    if (k == 6) return cudaErrorInvalidConfiguration;
+    if (k == nchoices) return cudaErrorInvalidConfiguration;
     P.NK = choices[k][0];
     P.NV = choices[k][1];
     P.NP = choices[k][2];
+    P.NQ = choices[k][3];
     const size_t smem = L.total + 1024;
     auto kfn = attn_tc_kernel<D, RP>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
