@@ -766,10 +766,10 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     }
 }
 
-constexpr int COMBINE_MAX_SEGS = 512;  // > num_ctas + 1 on any current GPU
-constexpr int COMBINE_REG_SEGS = 8;    // segments whose partial column is loaded up front
+constexpr int COMBINE_ROWS = 8;       // rows per combine CTA, one warp each
+constexpr int COMBINE_REG_SEGS = 8;   // segments whose partial row is loaded up front
 
-// Block-wide sum / max for blockDim.x <= 128 (at most 4 warps); red holds 4 slots.
+// Block-wide integer sum for blockDim.x <= 32 * COMBINE_ROWS; red holds one slot per warp.
 SV_DEV int block_sum_i(int v, int *red) {
     v = __reduce_add_sync(0xffffffffu, v);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
@@ -782,28 +782,26 @@ SV_DEV int block_sum_i(int v, int *red) {
 
 // Merge the partials of every unit that was split over several CTAs (a unit one
 // CTA covered whole was written by the attention kernel, and an invalid
-// sequence by its status warp). One CTA per (row of a unit, unit), one thread
-// per head dimension:
+// sequence by its status warp). One CTA per (COMBINE_ROWS rows, unit), one warp
+// per row, four head dimensions per lane:
 //   M = max_k m_k,  L = sum_k 2^(m_k - M) l_k,  out = sum_k 2^(m_k - M) O_k / L.
 // Launched as a programmatic dependent of the attention kernel, which lets it
 // launch only after its own wait on earlier work: the schedule is recomputed
 // from ctx_lens (complete by then) before this kernel waits, so once the
 // attention kernel completes one round of loads remains.
-__global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const AttnParams p) {
     griddep_launch_dependents();  // the next call's attention kernel may run its prologue
-    const int r = blockIdx.x, u = blockIdx.y, d = threadIdx.x, nt = blockDim.x;
+    const int u = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = p.D, RU = p.rows_unit;
     const int ups = p.Hkv * p.RC;
     const int b = u / ups, hr = u - b * ups;
     const int h = hr / p.RC, rc = hr - h * p.RC;
     const int rows = min(RU, p.R - rc * RU);
-    if (r >= rows) return;
-    __shared__ int red_i[4];
-    __shared__ float red_f[4];
-    __shared__ float sw[COMBINE_MAX_SEGS];
+    const int r = blockIdx.x * COMBINE_ROWS + warp;
+    __shared__ int red_i[COMBINE_ROWS];
     // the attention kernel's schedule: all tiles, those before sequence b, b's own
     int tot = 0, before = 0, own = 0;
-    for (int s = d; s < p.B; s += nt) {
+    for (int s = threadIdx.x; s < p.B; s += blockDim.x) {
         const int t = seq_tiles(p, s);
         tot += t;
         before += s < b ? t : 0;
@@ -812,7 +810,7 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
     tot = block_sum_i(tot, red_i);
     before = block_sum_i(before, red_i);
     const int Tb = block_sum_i(own, red_i);
-    if (Tb == 0) return;
+    if (Tb == 0 || r >= rows) return;
     const int total = ups * tot;
     const int W = (total + p.num_ctas - 1) / p.num_ctas;
     const int tpre = ups * before + hr * Tb;
@@ -820,55 +818,58 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(const AttnParams p) {
     if (n == 1) return;
     const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
-    const size_t slot_floats = slot_stride(RU, D);
-    const float *seg0 = p.ws_partial + (size_t)(u + first) * slot_floats;
+    const size_t sf = slot_stride(RU, D);
+    const float *seg0 = p.ws_partial + (size_t)(u + first) * sf;
+    const bool dl = lane < D / 4;  // this lane holds head dims 4*lane .. 4*lane+3
 
     griddep_wait();  // the partials are complete and visible
-    // one round of loads: this thread's column of the first partials, and the
-    // (m, l) of segment d
-    float ov[COMBINE_REG_SEGS];
+    // one round of loads: this lane's dims of the first partials, and segment lane's (m, l)
+    float4 ov[COMBINE_REG_SEGS];
 #pragma unroll
     for (int k = 0; k < COMBINE_REG_SEGS; ++k)
-        ov[k] = k < n ? __ldcg(seg0 + (size_t)k * slot_floats + (size_t)r * D + d) : 0.f;
+        ov[k] = (k < n && dl) ? __ldcg(reinterpret_cast<const float4 *>(seg0 + (size_t)k * sf + (size_t)r * D) + lane)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
     float mk = -INFINITY, lk = 0.f;
-    if (d < n) {
-        mk = __ldcg(seg0 + (size_t)d * slot_floats + (size_t)RU * D + r);
-        lk = __ldcg(seg0 + (size_t)d * slot_floats + (size_t)RU * D + RU + r);
+    if (lane < n) {
+        mk = __ldcg(seg0 + (size_t)lane * sf + (size_t)RU * D + r);
+        lk = __ldcg(seg0 + (size_t)lane * sf + (size_t)RU * D + RU + r);
     }
-    float m = mk;
-    for (int k = d + nt; k < n; k += nt) m = fmaxf(m, __ldcg(seg0 + (size_t)k * slot_floats + (size_t)RU * D + r));
-    m = warp_max(m);
-    if ((d & 31) == 0) red_f[d >> 5] = m;
-    __syncthreads();
-    float M = red_f[0];
-    for (int w = 1; w < (nt + 31) / 32; ++w) M = fmaxf(M, red_f[w]);
-    __syncthreads();
-    float lw = 0.f;
-    if (d < n) {
-        const float w = (mk == -INFINITY) ? 0.f : exp2f(mk - M);
-        sw[d] = w;
-        lw = w * lk;
+    float M = mk;
+    for (int k = lane + 32; k < n; k += 32) M = fmaxf(M, __ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r));
+    M = warp_max(M);
+    const float wl = lane < n ? exp2f(mk - M) : 0.f;  // an empty segment holds l = 0
+    float L = wl * lk;
+    for (int k = lane + 32; k < n; k += 32) {
+        const float *sg = seg0 + (size_t)k * sf + (size_t)RU * D;
+        L = fmaf(exp2f(__ldcg(sg + r) - M), __ldcg(sg + RU + r), L);
     }
-    for (int k = d + nt; k < n; k += nt) {
-        const float *sg = seg0 + (size_t)k * slot_floats + (size_t)RU * D;
-        const float mkk = __ldcg(sg + r);
-        const float w = (mkk == -INFINITY) ? 0.f : exp2f(mkk - M);
-        sw[k] = w;
-        lw = fmaf(w, __ldcg(sg + RU + r), lw);
-    }
-    lw = warp_sum(lw);
-    if ((d & 31) == 0) red_f[d >> 5] = lw;
-    __syncthreads();  // also publishes sw
-    float L = 0.f;
-    for (int w = 0; w < (nt + 31) / 32; ++w) L += red_f[w];
-    float acc = 0.f;
+    L = warp_sum(L);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int k = 0; k < COMBINE_REG_SEGS; ++k)
-        if (k < n) acc = fmaf(sw[k], ov[k], acc);
-    for (int k = COMBINE_REG_SEGS; k < n; ++k)
-        acc = fmaf(sw[k], __ldcg(seg0 + (size_t)k * slot_floats + (size_t)r * D + d), acc);
-    const __nv_bfloat16 o = __float2bfloat16_rn(L > 0.f ? acc / L : 0.f);
-    p.out[(((size_t)b * p.N + i) * p.Hq + hq) * D + d] = *reinterpret_cast<const uint16_t *>(&o);
+    for (int k = 0; k < COMBINE_REG_SEGS; ++k) {
+        const float w = __shfl_sync(0xffffffffu, wl, k);
+        if (k < n) {
+            acc.x = fmaf(w, ov[k].x, acc.x); acc.y = fmaf(w, ov[k].y, acc.y);
+            acc.z = fmaf(w, ov[k].z, acc.z); acc.w = fmaf(w, ov[k].w, acc.w);
+        }
+    }
+    for (int k = COMBINE_REG_SEGS; k < n; ++k) {
+        const float w = k < 32 ? __shfl_sync(0xffffffffu, wl, k)
+                               : exp2f(__ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r) - M);
+        if (dl) {
+            const float4 o = __ldcg(reinterpret_cast<const float4 *>(seg0 + (size_t)k * sf + (size_t)r * D) + lane);
+            acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
+        }
+    }
+    if (!dl) return;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    const __nv_bfloat162 o01 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+    const __nv_bfloat162 o23 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+    uint2 packed;
+    packed.x = *reinterpret_cast<const uint32_t *>(&o01);
+    packed.y = *reinterpret_cast<const uint32_t *>(&o23);
+    *reinterpret_cast<uint2 *>(p.out + (((size_t)b * p.N + i) * p.Hq + hq) * D + 4 * lane) = packed;
 }
 
 // ---------------------------------------------------------------------------
@@ -1025,7 +1026,8 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     const int RP = (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess) return e;
-    return launch_programmatic(attn_combine_kernel, dim3(RU, p.units), dim3(p.D), 0, stream, p);
+    return launch_programmatic(attn_combine_kernel, dim3((RU + COMBINE_ROWS - 1) / COMBINE_ROWS, p.units),
+                               dim3(32 * COMBINE_ROWS), 0, stream, p);
 }
 
 }  // namespace sv
