@@ -173,7 +173,7 @@ __host__ __device__ inline TcLayout tc_layout(int D, int RP, int NK, int NV, int
     L.p_bytes = (uint32_t)((RP + 63) / 64) * ATOM;
     L.off_bar = L.off_p + NP * L.p_bytes;
     const int nbar = 2 * NK + 2 * NV + 2 * 2 /*q*/ + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 * 2 /*o*/ + 1 /*done*/ +
-                     NWG /*wg*/;
+                     NWG /*wg*/ + NV /*vz*/;
     L.off_tp = L.off_bar + 8u * nbar;
     L.off_cl = L.off_tp + 4u * (B + 1);
     L.off_red = (L.off_cl + 4u * B + 15u) & ~15u;
@@ -232,6 +232,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     uint64_t *o_free = o_full + 2;     // [2] by unit parity: the unit's O buffer has been read out
     uint64_t *done_bar = o_free + 2;
     uint64_t *wg_bar = done_bar + 1;   // [NWG] warpgroup-local barriers
+    uint64_t *vz = wg_bar + NWG;       // [NV] the tile's V is ready for its PV (rows past ctx_len zeroed)
     int *TP = reinterpret_cast<int *>(base + L.off_tp);
     int *CL = reinterpret_cast<int *>(base + L.off_cl);
     float *red = reinterpret_cast<float *>(base + L.off_red);
@@ -259,6 +260,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         }
         for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], MATH_WARPS); mbar_init(&p_empty[i], 1); }
         mbar_init(done_bar, 1);
+        for (int s = 0; s < NV; ++s) mbar_init(&vz[s], 1);
         for (int g = 0; g < NWG; ++g) mbar_init(&wg_bar[g], WARPS_PER_WG);
         *abort_flag = 0;
         fence_barrier_init();
@@ -373,6 +375,30 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             if (p.status && lane == 0)
                 p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0);
         }
+        // ------------------- V rows past ctx_len -------------------
+        // Softmax gives keys past ctx_len p = 0, but 0 * NaN is NaN and those
+        // rows of the last page hold whatever the pool holds; they are zeroed
+        // here once the tile has landed, off the softmax path. Every tile is
+        // released to its PV through vz, after its V has landed, so this warp
+        // stays within one phase of the V ring.
+        TileInfo ti = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+        for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
+            const int s = lt % NV;
+            const uint32_t par = (lt / NV) & 1;
+            const bool landed = mbar_test(&v_full[s], par) || mbar_wait(&v_full[s], par, abort_flag, WAIT_LIMIT_NS);
+            if (!__all_sync(0xffffffffu, landed)) break;
+            const int k0 = max(0, CL[ti.b] - ti.j * TILE_KEYS);  // first key of the tile past ctx_len
+            if (k0 < TILE_KEYS) {
+                uint8_t *vt = base + s * L.tile_bytes;
+                for (int e = lane; e < (TILE_KEYS - k0) * 8 * nDA; e += 32) {
+                    const int key = k0 + e / (8 * nDA), rem = e - (key - k0) * (8 * nDA);
+                    reinterpret_cast<uint4 *>(vt + (rem >> 3) * ATOM + key * 128)[rem & 7] = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&vz[s]);
+        }
     } else if (warp == WARP_MMA) {
         // -------------------------- MMA issuer ----------------------------
         // Polls both queues and issues whichever product is ready: QK of the
@@ -421,6 +447,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     const int lup_n = newu ? lup + 1 : lup;
                     const int s = np % NV, pb = np % NP, ob = lup_n & 1;
                     if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&v_full[s], (np / NV) & 1) &&
+                        mbar_test(&vz[s], (np / NV) & 1) &&
                         (!newu || mbar_test(&o_free[ob], ((lup_n >> 1) & 1) ^ 1))) {
                         lup = lup_n;
                         tc_fence_after();
@@ -735,17 +762,6 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 uint4 *dst = reinterpret_cast<uint4 *>(pbuf + (cc >> 6) * ATOM + (ell >> 3) * 1024 +
                                                        (ell & 7) * 128 + ((chunk ^ (ell & 7)) << 4));
                 *dst = make_uint4(packed[c8 * 4], packed[c8 * 4 + 1], packed[c8 * 4 + 2], packed[c8 * 4 + 3]);
-            }
-            if (__any_sync(0xffffffffu, !valid) && wg == 0) {
-                // a key past ctx_len: its V row may hold anything (NaN) and P = 0 does not
-                // cancel it, so the row is zeroed once the tile's V has landed
-                if (!(ok = wait_w(&v_full[lt % NV], (lt / NV) & 1))) break;
-                if (!valid) {
-                    uint8_t *vrow = base + (lt % NV) * L.tile_bytes + ell * 128;
-                    for (int a = 0; a < nDA; ++a)
-                        for (int q = 0; q < 8; ++q)
-                            reinterpret_cast<uint4 *>(vrow + a * ATOM)[q] = make_uint4(0, 0, 0, 0);
-                }
             }
             fence_proxy_async_smem();
             warp_arrive(&p_full[pb]);
