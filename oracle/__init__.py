@@ -53,6 +53,8 @@ def lib() -> C.CDLL:
         L.orc_accept.restype = i32
         L.orc_inv_cdf.argtypes = [P, i32, f64, P]
         L.orc_inv_cdf.restype = i32
+        L.orc_kv_commit.argtypes = [i32] * 8 + [P] * 8
+        L.orc_kv_commit.restype = i32
         _lib = L
     return _lib
 
@@ -163,3 +165,31 @@ def inv_cdf(w: np.ndarray, u: float):
     gap = np.zeros(1, dtype=np.float64)
     x = lib().orc_inv_cdf(_p(a), a.size, float(u), _p(gap))
     return x, float(gap[0])
+
+
+def kv_commit(pools, block_table, ctx_lens, accept_len, accept_path, num_q_rows: int):
+    """KV commit after accept, in place on the numpy uint16 (bf16 bits) pools.
+
+    pools: list of (k_pool, v_pool) arrays [num_blocks][Hkv][bs][D], one pair per
+    layer. Returns (new_ctx_lens, flags)."""
+    k0 = pools[0][0]
+    num_blocks, Hkv, bs, D = k0.shape
+    tbl = np.ascontiguousarray(block_table, dtype=np.int32)
+    B, max_blocks = tbl.shape
+    lens = np.ascontiguousarray(ctx_lens, dtype=np.int32)
+    alen = np.ascontiguousarray(accept_len, dtype=np.int32)
+    N = int(num_q_rows)
+    path = np.ascontiguousarray(accept_path, dtype=np.int32).reshape(B, max(N - 1, 1)) if N > 1 else \
+        np.zeros((B, 1), dtype=np.int32)
+    for k, v in pools:
+        assert k.dtype == np.uint16 and v.dtype == np.uint16 and k.flags.c_contiguous and v.flags.c_contiguous
+    kp = (C.c_void_p * len(pools))(*[k.ctypes.data for k, _ in pools])
+    vp = (C.c_void_p * len(pools))(*[v.ctypes.data for _, v in pools])
+    new_lens = np.zeros(B, dtype=np.int32)
+    flags = np.zeros(B, dtype=np.int32)
+    rc = lib().orc_kv_commit(B, N, Hkv, D, bs, max_blocks, num_blocks, len(pools), C.cast(kp, C.c_void_p),
+                             C.cast(vp, C.c_void_p), _p(tbl), _p(lens), _p(alen), _p(path), _p(new_lens),
+                             _p(flags))
+    if rc:
+        raise ValueError(f"orc_kv_commit returned {rc}")
+    return new_lens, flags

@@ -416,3 +416,77 @@ int orc_inv_cdf(const double *w, int V, double u, double *gap)
 {
     return inv_cdf(w, V, u, gap);
 }
+
+/* ------------------------------------------------------------------------ */
+/* KV commit after accept                                                    */
+/* ------------------------------------------------------------------------ */
+/*
+ * After verification the cache keeps the last accepted token's row (the tree
+ * root, position C - N) and the accepted draft nodes; rejected drafts are
+ * dropped (TLT reading notes, "1. RL and SD": results computed on top of a
+ * rejected token are discarded; SRT review, "Speculative Rollout integration":
+ * the accepted path of the verified tree continues the sequence). The
+ * accepted nodes are compacted behind the root in path order:
+ *   K/V at position C - N + path[k]  ->  position C - N + 1 + k,  k < a,
+ *   new ctx_len = C - N + 1 + a,
+ * for every layer and KV head. Positions past the new length keep whatever
+ * they held. A chain's path is 1..a, so nothing moves.
+ * A sequence is left untouched (new ctx_len = ctx_len) and flagged when
+ * ctx_len is outside [N, max_blocks*bs] (bit 1), a page holding one of its N
+ * new positions has a block id outside the pool (bit 3), or accept_len is
+ * outside [0, N-1] or the path is not strictly increasing within [1, N-1]
+ * (bit 5).
+ * pools: num_layers (k, v) pairs of bf16 [num_blocks][Hkv][bs][D], in place.
+ */
+int orc_kv_commit(int B, int N, int Hkv, int D, int bs, int max_blocks, int num_blocks, int num_layers,
+                  uint16_t *const *k_pools, uint16_t *const *v_pools, const int32_t *block_table,
+                  const int32_t *ctx_lens, const int32_t *accept_len, const int32_t *accept_path,
+                  int32_t *new_ctx_lens, int32_t *flags)
+{
+    if (B < 0 || N < 1 || N > 64 || Hkv < 1 || D < 1 || bs < 1 || num_layers < 0) return -2;
+    uint16_t *row = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)D * 64);
+    if (!row) return -3;
+    for (int b = 0; b < B; ++b) {
+        const int C = ctx_lens[b];
+        int f = 0;
+        if (C < N || C > max_blocks * bs) f |= 2;
+        if (!f)
+            for (int t = C - N; t < C; ++t) {
+                const int blk = block_table[(size_t)b * max_blocks + t / bs];
+                if (blk < 0 || blk >= num_blocks) { f |= 8; break; }
+            }
+        const int a = accept_len[b];
+        if (a < 0 || a > N - 1) f |= 32;
+        else
+            for (int k = 0; k < a; ++k) {
+                const int node = accept_path[(size_t)b * (N > 1 ? N - 1 : 1) + k];
+                const int prev = k > 0 ? accept_path[(size_t)b * (N - 1) + k - 1] : 0;
+                if (node < 1 || node > N - 1 || node <= prev) { f |= 32; break; }
+            }
+        flags[b] = f;
+        if (f) { new_ctx_lens[b] = C; continue; }
+        new_ctx_lens[b] = C - N + 1 + a;
+        for (int l = 0; l < num_layers; ++l)
+            for (int kv = 0; kv < 2; ++kv) {
+                uint16_t *pool = kv ? v_pools[l] : k_pools[l];
+                for (int h = 0; h < Hkv; ++h) {
+                    /* gather every source row first, then write: a destination can be
+                     * another move's source */
+                    for (int k = 0; k < a; ++k) {
+                        const int t = C - N + accept_path[(size_t)b * (N - 1) + k];
+                        const int blk = block_table[(size_t)b * max_blocks + t / bs];
+                        memcpy(row + (size_t)k * D, pool + (((size_t)blk * Hkv + h) * bs + t % bs) * D,
+                               sizeof(uint16_t) * (size_t)D);
+                    }
+                    for (int k = 0; k < a; ++k) {
+                        const int t = C - N + 1 + k;
+                        const int blk = block_table[(size_t)b * max_blocks + t / bs];
+                        memcpy(pool + (((size_t)blk * Hkv + h) * bs + t % bs) * D, row + (size_t)k * D,
+                               sizeof(uint16_t) * (size_t)D);
+                    }
+                }
+            }
+    }
+    free(row);
+    return 0;
+}

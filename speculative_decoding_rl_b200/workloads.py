@@ -265,6 +265,29 @@ def make_accept_inputs(num_seqs: int, num_rows: int, vocab: int, seed: int, *,
                         q.contiguous(), d.contiguous(), float(temperature))
 
 
+def make_accept_paths(num_q_rows: int, parents: Optional[Sequence[int]], num_seqs: int, seed: int,
+                      max_len: Optional[int] = None):
+    """Seeded accepted paths of the shape the accept call returns: per sequence a
+    random walk from the root down the draft tree (a chain when parents is None),
+    stopping at a random depth. Returns (accept_len int32 [B], accept_path int32
+    [B][N-1], -1 after the end)."""
+    N = num_q_rows
+    par = list(parents) if parents is not None else [-1] + list(range(N - 1))
+    children = [[c for c in range(1, N) if par[c] == v] for v in range(N)]
+    rng = np.random.default_rng(seed)
+    alen = np.zeros(num_seqs, dtype=np.int32)
+    path = np.full((num_seqs, max(N - 1, 1)), -1, dtype=np.int32)
+    for b in range(num_seqs):
+        v, depth = 0, 0
+        target = int(rng.integers(0, N)) if max_len is None else int(max_len)
+        while depth < target and children[v]:
+            v = int(rng.choice(children[v]))
+            path[b, depth] = v
+            depth += 1
+        alen[b] = depth
+    return torch.from_numpy(alen), torch.from_numpy(path)
+
+
 # ---------------------------------------------------------------------------
 # The five workloads. Layer counts come from the public model configs of the
 # named model shapes and turn one layer's attention time into a verify step.
