@@ -426,6 +426,38 @@ def run_ours(args, world, rank, local):
         e2e = {"value": steps_total / e2e_elapsed, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h)}
 
+    # KV commit after accept (keep the root and the accepted nodes, compacted),
+    # over the distinct pools, with the last step's accept results; reported
+    # beside the verify step, which stays attention + accept
+    n_commit = min(layers, n_pools)
+    commit_layers = [(calls[i].k_pool, calls[i].v_pool) for i in range(n_commit)]
+    torch.cuda.synchronize()
+    alen_c = acc.accept_len.clone()  # the last accept call's results, as a pair
+    path_c = acc.path.clone() if acc.path is not None else torch.zeros((B, 1), dtype=torch.int32, device=dev)
+    from speculative_decoding_rl_b200.session import CommitCall
+    cc = CommitCall(calls[0].desc, commit_layers, calls[0].block_table, calls[0].ctx_lens, alen_c, path_c,
+                    device=str(dev))
+    cst = cc.status
+
+    def commit():
+        cc.run(stream)
+
+    for _ in range(2):
+        commit()
+    torch.cuda.synchronize()
+    c0, c1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c0.record(stream)
+    for _ in range(10):
+        commit()
+    c1.record(stream)
+    torch.cuda.synchronize()
+    a_host, p_host = alen_c.cpu().numpy(), path_c.cpu().numpy()
+    moved = sum(int(a_host[b]) for b in range(B)
+                if any(int(p_host[b, k]) != k + 1 for k in range(int(a_host[b]))))
+    commit_info = {"call_ms": c0.elapsed_time(c1) / 10, "layers": n_commit,
+                   "bytes_moved": 2 * 2 * moved * a0.num_kv_heads * D * 2 * n_commit,
+                   "flags_clear": bool((cst == 0).all().item())}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, ta, tc, sample = oracle_sample(w, a0, acc_in, layers, args.cpu_sample_seconds)
@@ -453,7 +485,7 @@ def run_ours(args, world, rank, local):
                          "kernel": "sv_verify_attention call: attn_tc_kernel + attn_combine_kernel",
                          "algorithmic_bytes_per_call": alg_bytes, "peak_source": peak_kind},
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * (2 * layers + 1),
-            "clocks": clocks, "parity": parity,
+            "clocks": clocks, "parity": parity, "kv_commit": commit_info,
         }
         print(json.dumps(line), flush=True)
 

@@ -67,6 +67,8 @@ typedef enum {
 #define SV_FLAG_BAD_TOKEN   4  /* accept: a draft token outside [0, vocab) */
 #define SV_FLAG_BAD_BLOCK   8  /* attention: a block id outside [0, num_blocks) */
 #define SV_FLAG_TIMEOUT    16  /* attention: a bounded device-side wait gave up; outputs invalid */
+#define SV_FLAG_BAD_PATH   32  /* kv commit: accept_len outside [0, N-1] or a path not strictly
+                                  increasing within [1, N-1] */
 
 /* ------------------------------------------------------------------------
  * Verify attention
@@ -165,6 +167,49 @@ SV_API sv_status sv_accept(const sv_accept_desc *desc, const float *target_logit
                     const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
                     int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
                     int32_t *status_flags, void *stream);
+
+/* ------------------------------------------------------------------------
+ * KV commit after accept
+ * ------------------------------------------------------------------------
+ * After verification the cache keeps the row of the last accepted token (the
+ * tree root, position ctx_len - N) and the accepted draft nodes, and drops the
+ * rest: results computed on top of a rejected draft are discarded (TLT reading
+ * notes, "1. RL and SD"), and the verified tree's accepted path continues the
+ * sequence (SRT review, "Speculative Rollout integration"). The accepted
+ * nodes are compacted behind the root in path order, in every layer and KV
+ * head:
+ *   K/V at position C - N + accept_path[b][k]  ->  position C - N + 1 + k,
+ *   new_ctx_lens[b] = C - N + 1 + accept_len[b]          (C = ctx_lens[b]).
+ * A chain's path is 1..a, so nothing moves and only the length changes.
+ * Positions past the new length keep what they held and the block table is
+ * not changed: pages past ceil(new_ctx_len / 16) are the caller's to reuse.
+ *   desc          the attention descriptor of the verify call (num_q_heads is
+ *                 unused; the pools' shape is [num_blocks][Hkv][16][D])
+ *   layers        HOST array of num_layers {k_pool, v_pool} device pointers,
+ *                 written in place; 1 <= num_layers <= SV_COMMIT_MAX_LAYERS
+ *   block_table, ctx_lens   as for sv_verify_attention
+ *   accept_len    int32 [B], accept_path int32 [B][N-1] (-1 padded), as
+ *                 sv_accept returns them
+ *   new_ctx_lens  int32 [B] out; status_flags int32 [B] or NULL
+ * A sequence is left untouched (new_ctx_len = ctx_len) and flagged when its
+ * ctx_len is outside [N, max_blocks*16] (SV_FLAG_BAD_CONTEXT), a page of its N
+ * new positions has a block id outside the pool (SV_FLAG_BAD_BLOCK), or its
+ * accept_len or path is malformed (SV_FLAG_BAD_PATH). Every source row is read
+ * before any row is written, so overlapping moves are safe. Limits: D a
+ * multiple of 8 up to 256, N <= 64. Pools 16-byte aligned.
+ * The pages have no interface for this step; its arguments follow the verify
+ * and accept calls whose results it applies.
+ */
+#define SV_COMMIT_MAX_LAYERS 128
+typedef struct {
+    void *k_pool;                /* bf16 [num_blocks][Hkv][16][D], written in place */
+    void *v_pool;
+} sv_kv_layer;
+
+SV_API sv_status sv_kv_commit(const sv_attn_desc *desc, int32_t num_layers, const sv_kv_layer *layers,
+                              const int32_t *block_table, const int32_t *ctx_lens, const int32_t *accept_len,
+                              const int32_t *accept_path, int32_t *new_ctx_lens, int32_t *status_flags,
+                              void *stream);
 
 /* ------------------------------------------------------------------------
  * Verify attention without a workspace argument

@@ -15,8 +15,9 @@ import os
 from typing import Optional, Sequence
 
 __all__ = [
-    "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc",
+    "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc", "SvKVLayer",
     "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
+    "sv_kv_commit", "make_kv_layers",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
 ]
@@ -30,6 +31,8 @@ SV_FLAG_BAD_CONTEXT = 2
 SV_FLAG_BAD_TOKEN = 4
 SV_FLAG_BAD_BLOCK = 8
 SV_FLAG_TIMEOUT = 16
+SV_FLAG_BAD_PATH = 32
+SV_COMMIT_MAX_LAYERS = 128
 SV_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -46,6 +49,10 @@ class SvAttnDesc(C.Structure):
 
 
 class SvPagedKV(C.Structure):
+    _fields_ = [("k_pool", C.c_void_p), ("v_pool", C.c_void_p)]
+
+
+class SvKVLayer(C.Structure):
     _fields_ = [("k_pool", C.c_void_p), ("v_pool", C.c_void_p)]
 
 
@@ -69,6 +76,8 @@ def _load() -> C.CDLL:
     L.sv_verify_attention_noalloc.restype = C.c_int
     L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P]
     L.sv_accept.restype = C.c_int
+    L.sv_kv_commit.argtypes = [C.POINTER(SvAttnDesc), i32, C.POINTER(SvKVLayer), P, P, P, P, P, P, P]
+    L.sv_kv_commit.restype = C.c_int
     L.sv_status_string.argtypes = [C.c_int]
     L.sv_status_string.restype = C.c_char_p
     L.sv_last_error.argtypes = []
@@ -162,6 +171,20 @@ def sv_accept(desc: SvAcceptDesc, target_logits, draft_probs, draft_tokens, temp
     _check(_L().sv_accept(C.byref(desc), _ptr(target_logits), _ptr(draft_probs), _ptr(draft_tokens),
                           float(temperature), int(philox_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(accept_len),
                           _ptr(next_token), _ptr(accept_path), _ptr(status_flags), _stream(stream)))
+
+
+def sv_kv_commit(desc: SvAttnDesc, layers, block_table, ctx_lens, accept_len, accept_path, new_ctx_lens,
+                 status_flags=None, stream=None) -> None:
+    """layers: a sequence of (k_pool, v_pool) pairs (tensors or device addresses), one per
+    layer, or an array built once with ``make_kv_layers``."""
+    arr = layers if isinstance(layers, C.Array) else make_kv_layers(layers)
+    _check(_L().sv_kv_commit(C.byref(desc), len(layers), arr, _ptr(block_table), _ptr(ctx_lens), _ptr(accept_len),
+                             _ptr(accept_path), _ptr(new_ctx_lens), _ptr(status_flags), _stream(stream)))
+
+
+def make_kv_layers(layers) -> C.Array:
+    """The SvKVLayer array of sv_kv_commit, built once for repeated calls."""
+    return (SvKVLayer * len(layers))(*[SvKVLayer(_ptr(k), _ptr(v)) for k, v in layers])
 
 
 def make_accept_desc(num_seqs: int, num_rows: int, vocab: int,

@@ -170,4 +170,54 @@ sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const f
     return SV_OK;
 }
 
+sv_status sv_kv_commit(const sv_attn_desc *d, int32_t num_layers, const sv_kv_layer *layers,
+                       const int32_t *block_table, const int32_t *ctx_lens, const int32_t *accept_len,
+                       const int32_t *accept_path, int32_t *new_ctx_lens, int32_t *status_flags, void *stream) {
+    if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
+    if (d->num_seqs < 0) return fail(SV_ERR_INVALID_ARG, "num_seqs < 0");
+    if (d->num_q_rows < 1 || d->num_q_rows > 64) return fail(SV_ERR_INVALID_ARG, "num_q_rows must be in [1, 64]");
+    if (d->num_kv_heads < 1 || d->num_kv_heads > 65535) return fail(SV_ERR_INVALID_ARG, "num_kv_heads must be in [1, 65535]");
+    if (d->head_dim < 8 || d->head_dim > 256 || d->head_dim % 8)
+        return fail(SV_ERR_UNSUPPORTED, "head_dim must be a multiple of 8 in [8, 256]");
+    if (d->block_size != sv::PAGE) return fail(SV_ERR_UNSUPPORTED, "block_size must be 16");
+    if (d->max_blocks_per_seq < 1) return fail(SV_ERR_INVALID_ARG, "max_blocks_per_seq < 1");
+    if (d->num_blocks < 1) return fail(SV_ERR_INVALID_ARG, "num_blocks < 1");
+    if ((long long)d->max_blocks_per_seq * sv::PAGE > (1LL << 30)) return fail(SV_ERR_UNSUPPORTED, "context too long");
+    if (num_layers < 1 || num_layers > SV_COMMIT_MAX_LAYERS)
+        return fail(SV_ERR_INVALID_ARG, "num_layers must be in [1, %d]", SV_COMMIT_MAX_LAYERS);
+    if (!layers) return fail(SV_ERR_INVALID_ARG, "layers is NULL");
+    for (int l = 0; l < num_layers; ++l)
+        if (!layers[l].k_pool || !layers[l].v_pool || !aligned(layers[l].k_pool, 16) || !aligned(layers[l].v_pool, 16))
+            return fail(SV_ERR_INVALID_ARG, "layer %d: pool NULL or not 16-byte aligned", l);
+    if (d->num_seqs == 0) return SV_OK;
+    if (!block_table || !ctx_lens || !accept_len || !new_ctx_lens)
+        return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (d->num_q_rows > 1 && !accept_path) return fail(SV_ERR_INVALID_ARG, "accept_path is NULL");
+    if (!aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(accept_len, 4) || !aligned(new_ctx_lens, 4) ||
+        (accept_path && !aligned(accept_path, 4)) || (status_flags && !aligned(status_flags, 4)))
+        return fail(SV_ERR_INVALID_ARG, "misaligned pointer");
+    sv::CommitLaunch c;
+    memset(&c, 0, sizeof c);
+    c.block_table = block_table;
+    c.ctx_lens = ctx_lens;
+    c.accept_len = accept_len;
+    c.accept_path = accept_path;
+    c.new_ctx = new_ctx_lens;
+    c.status = status_flags;
+    c.B = d->num_seqs;
+    c.N = d->num_q_rows;
+    c.Hkv = d->num_kv_heads;
+    c.D = d->head_dim;
+    c.max_blocks = d->max_blocks_per_seq;
+    c.num_blocks = d->num_blocks;
+    c.L = num_layers;
+    for (int l = 0; l < num_layers; ++l) {
+        c.k[l] = static_cast<uint16_t *>(layers[l].k_pool);
+        c.v[l] = static_cast<uint16_t *>(layers[l].v_pool);
+    }
+    cudaError_t e = sv::launch_kv_commit(c, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SV_ERR_CUDA, "kv commit launch: %s", cudaGetErrorString(e));
+    return SV_OK;
+}
+
 }  // extern "C"

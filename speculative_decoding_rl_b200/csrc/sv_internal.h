@@ -62,6 +62,16 @@ void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc);
 int attention_num_ctas();
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
 
+// ------------------------------- kv commit ----------------------------------
+struct CommitLaunch {
+    const int32_t *block_table, *ctx_lens, *accept_len, *accept_path;
+    int32_t *new_ctx, *status;
+    int B, N, Hkv, D, max_blocks, num_blocks, L;
+    uint16_t *k[SV_COMMIT_MAX_LAYERS];
+    uint16_t *v[SV_COMMIT_MAX_LAYERS];
+};
+cudaError_t launch_kv_commit(const CommitLaunch &c, cudaStream_t stream);
+
 // Sets the text sv_last_error() returns on the calling thread.
 void record_error(const char *msg);
 

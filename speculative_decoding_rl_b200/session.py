@@ -1,4 +1,4 @@
-"""Device-resident call objects for the two verify-step entry points.
+"""Device-resident call objects for the verify-step entry points and the KV commit.
 
 Each object owns the device buffers of one call (inputs copied once with
 torch, outputs, workspace) and ``run()`` makes exactly one C-ABI call on the
@@ -11,8 +11,8 @@ from typing import Optional
 
 import torch
 
-from . import (SvAttnDesc, SvPagedKV, make_accept_desc, sv_accept, sv_verify_attention,
-               sv_verify_attention_workspace_size)
+from . import (SvAttnDesc, SvPagedKV, make_accept_desc, make_kv_layers, sv_accept, sv_kv_commit,
+               sv_verify_attention, sv_verify_attention_workspace_size)
 
 
 class AttentionCall:
@@ -65,3 +65,23 @@ class AcceptCall:
                   self.drafts if self.drafts.numel() else None, self.temperature, self.seed,
                   self.accept_len, self.next_token, self.path, self.status, stream)
         return self.accept_len, self.next_token
+
+
+class CommitCall:
+    """KV commit after accept over a fixed set of layers' pools (arguments prepared once)."""
+
+    def __init__(self, desc, layers, block_table, ctx_lens, accept_len, accept_path, device: str = "cuda"):
+        dev = torch.device(device)
+        B = desc.num_seqs
+        self.desc = desc
+        self.layers = layers
+        self._arr = make_kv_layers(layers)
+        self.block_table, self.ctx_lens = block_table, ctx_lens
+        self.accept_len, self.accept_path = accept_len, accept_path
+        self.new_ctx_lens = torch.empty(B, dtype=torch.int32, device=dev)
+        self.status = torch.empty(B, dtype=torch.int32, device=dev)
+
+    def run(self, stream=None):
+        sv_kv_commit(self.desc, self._arr, self.block_table, self.ctx_lens, self.accept_len, self.accept_path,
+                     self.new_ctx_lens, self.status, stream)
+        return self.new_ctx_lens

@@ -118,3 +118,29 @@ def test_accept_requires_outputs_and_drafts():
     with pytest.raises(sv.SvError) as e:
         sv.sv_accept(desc, 16, 16, 16, 1.0, 0, None, 16, None, None, stream=0)
     assert e.value.status == sv.SV_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kw,layers,status", [
+    (dict(num_q_rows=0), 1, 1), (dict(num_q_rows=65), 1, 1), (dict(head_dim=12), 1, 2),
+    (dict(head_dim=264), 1, 2), (dict(block_size=32), 1, 2), (dict(num_kv_heads=0), 1, 1),
+    (dict(num_blocks=0), 1, 1), ({}, 0, 1), ({}, 129, 1),
+])
+def test_kv_commit_rejects_bad_arguments(kw, layers, status):
+    base = dict(num_seqs=2, num_q_rows=5, num_q_heads=4, num_kv_heads=2, head_dim=128, block_size=16,
+                max_blocks_per_seq=4, num_blocks=8)
+    base.update(kw)
+    d = sv.SvAttnDesc(*[base[k] for k in ("num_seqs", "num_q_rows", "num_q_heads", "num_kv_heads", "head_dim",
+                                          "block_size", "max_blocks_per_seq", "num_blocks")])
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_kv_commit(d, [(256, 512)] * layers, 64, 64, 64, 64, 64)
+    assert e.value.status == status
+
+
+def test_kv_commit_rejects_null_and_misaligned_pointers():
+    d = sv.SvAttnDesc(2, 5, 4, 2, 128, 16, 4, 8)
+    for layers, args in [([(256, 8)], (64, 64, 64, 64, 64)), ([(256, 512)], (0, 64, 64, 64, 64)),
+                         ([(256, 512)], (64, 64, 64, 0, 64)), ([(256, 512)], (64, 66, 64, 64, 64))]:
+        with pytest.raises(sv.SvError) as e:
+            sv.sv_kv_commit(d, layers, *args)
+        assert e.value.status == 1
+    sv.sv_kv_commit(sv.SvAttnDesc(0, 5, 4, 2, 128, 16, 4, 8), [(256, 512)], 0, 0, 0, 0, 0)  # no sequences
