@@ -212,6 +212,113 @@ SV_API sv_status sv_kv_commit(const sv_attn_desc *desc, int32_t num_layers, cons
                               void *stream);
 
 /* ------------------------------------------------------------------------
+ * Host speculative-decoding controller
+ * ------------------------------------------------------------------------
+ * Host logic (no GPU work) that decides, for each decode step of a batch,
+ * whether to speculate, how many drafts to verify and which drafter to use,
+ * from costs measured with this library and the acceptance it observes:
+ *  - elastic enable: no speculation while more than elastic_max_batch
+ *    requests are active (TLT reading notes, "Elastic enable");
+ *  - roofline toggle: speculate only when a verify step is expected to
+ *    advance more tokens per millisecond than a plain decode step. The
+ *    target's forward pass over T tokens costs max(weight bytes / HBM rate,
+ *    T x flops per token / tensor rate) (memory-bound at small T, compute-bound
+ *    at large T), plus the measured verify-path cost of the bucket
+ *    (EfficientRollout, "System-aware SD toggle policy");
+ *  - draft length, either acceptance-aware: the gamma maximising expected
+ *    tokens per millisecond, sum_{k<=gamma} beta^k per sequence, under a
+ *    running per-token acceptance estimate beta (EfficientRollout,
+ *    "Acceptance-aware draft-length adaptation"); or BEG-MAB: per batch
+ *    bucket, the draft length with the best median of accepted tokens per
+ *    millisecond over a recent window, with occasional random exploration
+ *    (TLT reading notes, "BEG-MAB");
+ *  - drafter: timing_guard between a weight-free history drafter and a model
+ *    drafter, per batch bucket, with the History Tree PR's defaults
+ *    (sv_ctl_default_config) for EMA weight, switch margin, probe length,
+ *    comparison delay and cooldown ("dynamic_rl default policy timing_guard").
+ * The pages give no interface for this; the structures below carry what those
+ * policies need. A controller object is not thread-safe.
+ */
+#define SV_CTL_GAMMA_ACCEPTANCE 0   /* draft length from the acceptance estimate */
+#define SV_CTL_GAMMA_MAB        1   /* draft length from BEG-MAB per bucket */
+#define SV_DRAFTER_NONE    0
+#define SV_DRAFTER_HISTORY 1        /* weight-free drafts from earlier rollouts */
+#define SV_DRAFTER_MODEL   2        /* a draft model (EAGLE-style head, small model) */
+#define SV_CTL_MAX_BUCKETS 64
+#define SV_CTL_MAX_GAMMA   63
+
+typedef struct {
+    /* target forward pass (roofline) */
+    double target_weight_bytes;      /* bytes of target weights one forward pass reads */
+    double target_flops_per_token;   /* ~2 x target parameters */
+    double hbm_gbs;                  /* HBM GB/s */
+    double tensor_tflops;            /* dense tensor TFLOP/s */
+    double model_draft_ms;           /* model drafter: ms per drafted position (whole batch) */
+    double history_draft_ms;         /* history drafter: ms per step (lookup) */
+    /* verify-path cost measured with this library, per batch bucket */
+    int32_t num_buckets;             /* 1..SV_CTL_MAX_BUCKETS */
+    int32_t bucket_max_batch[SV_CTL_MAX_BUCKETS];   /* inclusive upper batch size, increasing */
+    int32_t gamma_max;               /* draft lengths 1..gamma_max considered */
+    const double *verify_ms;         /* HOST [num_buckets][gamma_max+1]: all layers' attention + accept at
+                                        gamma drafts; index 0 = plain decode (one row per sequence) */
+    /* policies */
+    int32_t elastic_max_batch;       /* 0 = no limit */
+    int32_t gamma_policy;            /* SV_CTL_GAMMA_* */
+    double accept_prior;             /* initial per-token acceptance estimate, in (0, 1) */
+    double accept_decay;             /* per-step decay of the acceptance counts, in [0, 1) */
+    int32_t mab_window;              /* BEG-MAB: recent steps kept per (bucket, gamma) */
+    double mab_explore;              /* BEG-MAB: probability of a random draft length */
+    uint64_t seed;                   /* exploration random numbers */
+    /* timing_guard */
+    int32_t use_model_drafter;       /* 0: history drafter only */
+    int32_t history_upper_batch;     /* history drafter only below this batch size */
+    int32_t model_max_batch;         /* model drafter considered at batch <= this */
+    int32_t model_probe_max_batch;   /* a probe of the model drafter starts only at batch <= this */
+    int32_t history_warmup_records;  /* history records before the history cache counts as warm */
+    int32_t model_cold_start_guard;  /* no model drafter before the history cache is warm */
+    int32_t compare_after_steps;     /* history steps in a bucket before the model drafter is probed */
+    int32_t model_probe_steps;       /* steps of one probe */
+    double score_ema_alpha;          /* weight of a new tokens/ms sample in a branch's score */
+    double switch_margin;            /* the model drafter needs score > history score x margin */
+    int32_t cooldown_steps;          /* steps on history after a bad probe */
+    int32_t max_cooldown_steps;
+    double cooldown_growth;          /* cooldown multiplier after consecutive bad probes */
+    double bad_step_ratio;           /* a model step below history score x ratio is a bad step */
+} sv_ctl_config;
+
+typedef struct {
+    int32_t speculate;               /* 0: plain decode step */
+    int32_t gamma;                   /* drafts per sequence (0 when not speculating) */
+    int32_t drafter;                 /* SV_DRAFTER_* */
+    int32_t bucket;                  /* batch bucket index */
+    double expected_tokens_per_ms;   /* the model's estimate for the chosen step */
+} sv_ctl_decision;
+
+typedef struct {
+    int32_t batch;                   /* sequences in the step */
+    int32_t gamma;                   /* drafts per sequence verified (0: plain step) */
+    int32_t drafter;                 /* SV_DRAFTER_* used */
+    int64_t accepted_drafts;         /* sum of accept_len over the batch */
+    int64_t rejections;              /* sequences whose accept_len < gamma */
+    double step_ms;                  /* measured time of the whole step */
+} sv_ctl_step;
+
+typedef struct sv_ctl sv_ctl;
+
+/* The History Tree PR's timing_guard defaults and neutral values for the rest. */
+SV_API void sv_ctl_default_config(sv_ctl_config *config);
+/* NULL with sv_last_error set on an invalid config; verify_ms is copied. */
+SV_API sv_ctl *sv_ctl_create(const sv_ctl_config *config);
+SV_API void sv_ctl_destroy(sv_ctl *ctl);
+/* Decision for a step of `batch` active requests with `history_records`
+ * records in the history drafter's cache. */
+SV_API sv_status sv_ctl_decide(sv_ctl *ctl, int32_t batch, int32_t history_records, sv_ctl_decision *out);
+/* Feed back a finished step (the decision it followed may differ: the caller decides). */
+SV_API sv_status sv_ctl_observe(sv_ctl *ctl, const sv_ctl_step *step);
+/* Current per-token acceptance estimate. */
+SV_API double sv_ctl_acceptance(const sv_ctl *ctl);
+
+/* ------------------------------------------------------------------------
  * Verify attention without a workspace argument
  * ------------------------------------------------------------------------
  * The source pages have no counterpart to this call; it exists for callers

@@ -17,7 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc", "SvKVLayer",
     "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
-    "sv_kv_commit", "make_kv_layers",
+    "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
 ]
@@ -33,6 +33,9 @@ SV_FLAG_BAD_BLOCK = 8
 SV_FLAG_TIMEOUT = 16
 SV_FLAG_BAD_PATH = 32
 SV_COMMIT_MAX_LAYERS = 128
+SV_CTL_GAMMA_ACCEPTANCE, SV_CTL_GAMMA_MAB = 0, 1
+SV_DRAFTER_NONE, SV_DRAFTER_HISTORY, SV_DRAFTER_MODEL = 0, 1, 2
+SV_CTL_MAX_BUCKETS = 64
 SV_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -54,6 +57,33 @@ class SvPagedKV(C.Structure):
 
 class SvKVLayer(C.Structure):
     _fields_ = [("k_pool", C.c_void_p), ("v_pool", C.c_void_p)]
+
+
+class SvCtlConfig(C.Structure):
+    _fields_ = [("target_weight_bytes", C.c_double), ("target_flops_per_token", C.c_double),
+                ("hbm_gbs", C.c_double), ("tensor_tflops", C.c_double), ("model_draft_ms", C.c_double),
+                ("history_draft_ms", C.c_double), ("num_buckets", C.c_int32),
+                ("bucket_max_batch", C.c_int32 * SV_CTL_MAX_BUCKETS), ("gamma_max", C.c_int32),
+                ("verify_ms", C.POINTER(C.c_double)), ("elastic_max_batch", C.c_int32),
+                ("gamma_policy", C.c_int32), ("accept_prior", C.c_double), ("accept_decay", C.c_double),
+                ("mab_window", C.c_int32), ("mab_explore", C.c_double), ("seed", C.c_uint64),
+                ("use_model_drafter", C.c_int32), ("history_upper_batch", C.c_int32),
+                ("model_max_batch", C.c_int32), ("model_probe_max_batch", C.c_int32),
+                ("history_warmup_records", C.c_int32), ("model_cold_start_guard", C.c_int32),
+                ("compare_after_steps", C.c_int32), ("model_probe_steps", C.c_int32),
+                ("score_ema_alpha", C.c_double), ("switch_margin", C.c_double), ("cooldown_steps", C.c_int32),
+                ("max_cooldown_steps", C.c_int32), ("cooldown_growth", C.c_double),
+                ("bad_step_ratio", C.c_double)]
+
+
+class SvCtlDecision(C.Structure):
+    _fields_ = [("speculate", C.c_int32), ("gamma", C.c_int32), ("drafter", C.c_int32), ("bucket", C.c_int32),
+                ("expected_tokens_per_ms", C.c_double)]
+
+
+class SvCtlStep(C.Structure):
+    _fields_ = [("batch", C.c_int32), ("gamma", C.c_int32), ("drafter", C.c_int32),
+                ("accepted_drafts", C.c_int64), ("rejections", C.c_int64), ("step_ms", C.c_double)]
 
 
 class SvAcceptDesc(C.Structure):
@@ -78,6 +108,18 @@ def _load() -> C.CDLL:
     L.sv_accept.restype = C.c_int
     L.sv_kv_commit.argtypes = [C.POINTER(SvAttnDesc), i32, C.POINTER(SvKVLayer), P, P, P, P, P, P, P]
     L.sv_kv_commit.restype = C.c_int
+    L.sv_ctl_default_config.argtypes = [C.POINTER(SvCtlConfig)]
+    L.sv_ctl_default_config.restype = None
+    L.sv_ctl_create.argtypes = [C.POINTER(SvCtlConfig)]
+    L.sv_ctl_create.restype = C.c_void_p
+    L.sv_ctl_destroy.argtypes = [C.c_void_p]
+    L.sv_ctl_destroy.restype = None
+    L.sv_ctl_decide.argtypes = [C.c_void_p, i32, i32, C.POINTER(SvCtlDecision)]
+    L.sv_ctl_decide.restype = C.c_int
+    L.sv_ctl_observe.argtypes = [C.c_void_p, C.POINTER(SvCtlStep)]
+    L.sv_ctl_observe.restype = C.c_int
+    L.sv_ctl_acceptance.argtypes = [C.c_void_p]
+    L.sv_ctl_acceptance.restype = C.c_double
     L.sv_status_string.argtypes = [C.c_int]
     L.sv_status_string.restype = C.c_char_p
     L.sv_last_error.argtypes = []
@@ -185,6 +227,54 @@ def sv_kv_commit(desc: SvAttnDesc, layers, block_table, ctx_lens, accept_len, ac
 def make_kv_layers(layers) -> C.Array:
     """The SvKVLayer array of sv_kv_commit, built once for repeated calls."""
     return (SvKVLayer * len(layers))(*[SvKVLayer(_ptr(k), _ptr(v)) for k, v in layers])
+
+
+def default_ctl_config() -> SvCtlConfig:
+    c = SvCtlConfig()
+    _L().sv_ctl_default_config(C.byref(c))
+    return c
+
+
+class SdController:
+    """The host speculative-decoding controller (sv_ctl_*): decide() before a
+    step, observe() after it. verify_ms: [num_buckets][gamma_max + 1] measured
+    verify-path milliseconds (index 0: a plain decode step)."""
+
+    def __init__(self, config: SvCtlConfig, bucket_max_batch: Sequence[int], verify_ms):
+        import numpy as np
+        v = np.ascontiguousarray(verify_ms, dtype=np.float64)
+        config.num_buckets = len(bucket_max_batch)
+        for i, b in enumerate(bucket_max_batch):
+            config.bucket_max_batch[i] = int(b)
+        config.gamma_max = v.shape[1] - 1
+        config.verify_ms = v.ctypes.data_as(C.POINTER(C.c_double))
+        self._h = _L().sv_ctl_create(C.byref(config))
+        if not self._h:
+            raise SvError(SV_ERR_INVALID_ARG, sv_last_error())
+
+    def decide(self, batch: int, history_records: int = 1) -> SvCtlDecision:
+        d = SvCtlDecision()
+        _check(_L().sv_ctl_decide(self._h, int(batch), int(history_records), C.byref(d)))
+        return d
+
+    def observe(self, batch: int, gamma: int, drafter: int, accepted_drafts: int, rejections: int,
+                step_ms: float) -> None:
+        s = SvCtlStep(int(batch), int(gamma), int(drafter), int(accepted_drafts), int(rejections), float(step_ms))
+        _check(_L().sv_ctl_observe(self._h, C.byref(s)))
+
+    def acceptance(self) -> float:
+        return _L().sv_ctl_acceptance(self._h)
+
+    def close(self) -> None:
+        if self._h:
+            _L().sv_ctl_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def make_accept_desc(num_seqs: int, num_rows: int, vocab: int,
