@@ -55,6 +55,8 @@ def lib() -> C.CDLL:
         L.orc_inv_cdf.restype = i32
         L.orc_kv_commit.argtypes = [i32] * 8 + [P] * 8
         L.orc_kv_commit.restype = i32
+        L.orc_history_draft.argtypes = [i32] * 7 + [P] * 10
+        L.orc_history_draft.restype = i32
         _lib = L
     return _lib
 
@@ -193,3 +195,26 @@ def kv_commit(pools, block_table, ctx_lens, accept_len, accept_path, num_q_rows:
     if rc:
         raise ValueError(f"orc_kv_commit returned {rc}")
     return new_lens, flags
+
+
+def history_draft(history_tokens, history_lens, history_reward, history_group, seq_tokens, seq_lens,
+                  seq_group, key_len: int, gamma: int, vocab: int = 0):
+    """Weight-free drafts from earlier responses. Returns (drafts [B][gamma],
+    draft_len [B], one-hot probs [B][gamma][vocab] or None)."""
+    ht = np.ascontiguousarray(history_tokens, dtype=np.int32)
+    st = np.ascontiguousarray(seq_tokens, dtype=np.int32)
+    H, hs = ht.shape
+    B, ss = st.shape
+    hl = np.ascontiguousarray(history_lens, dtype=np.int32)
+    hr = np.ascontiguousarray(history_reward, dtype=np.float32)
+    hg = np.ascontiguousarray(history_group, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    sg = np.ascontiguousarray(seq_group, dtype=np.int32)
+    drafts = np.zeros((B, gamma), dtype=np.int32)
+    dlen = np.zeros(B, dtype=np.int32)
+    probs = np.zeros((B, gamma, vocab), dtype=np.float32) if vocab > 0 else None
+    rc = lib().orc_history_draft(B, H, hs, ss, int(key_len), int(gamma), int(vocab), _p(ht), _p(hl), _p(hr),
+                                 _p(hg), _p(st), _p(sl), _p(sg), _p(drafts), _p(dlen), _p(probs))
+    if rc:
+        raise ValueError(f"orc_history_draft returned {rc}")
+    return drafts, dlen, probs

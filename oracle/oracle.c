@@ -490,3 +490,64 @@ int orc_kv_commit(int B, int N, int Hkv, int D, int bs, int max_blocks, int num_
     free(row);
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Weight-free drafts from earlier rollouts                                  */
+/* ------------------------------------------------------------------------ */
+/*
+ * History drafts (History Tree PR: drafts taken from earlier rollouts' high
+ * reward responses of the same prompt, with a global fallback; the SRT review's
+ * tree cache looks a sequence's prefix up in earlier rollouts). For sequence b
+ * the key is its last K tokens. A candidate is a response h and a position p
+ * with history[h][p..p+K-1] == key and at least one token after the key. The
+ * first pass considers responses of the sequence's group; when none matches,
+ * a second pass considers every response. The chosen candidate has the
+ * highest reward, then the lowest h, then the lowest p. Drafts are the up to
+ * gamma tokens after the key (draft_len), padded with token 0; a sequence
+ * shorter than K, or without a candidate, gets draft_len 0 and all padding.
+ * When probs is given (vocab > 0) each of the gamma rows is one-hot at its
+ * draft token.
+ */
+int orc_history_draft(int B, int H, int hstride, int sstride, int K, int gamma, int vocab,
+                      const int32_t *htok, const int32_t *hlen, const float *hreward, const int32_t *hgroup,
+                      const int32_t *stok, const int32_t *slen, const int32_t *sgroup,
+                      int32_t *drafts, int32_t *draft_len, float *probs)
+{
+    if (B < 0 || H < 0 || K < 1 || gamma < 1 || vocab < 0) return -2;
+    for (int b = 0; b < B; ++b) {
+        int best_h = -1, best_p = -1;
+        const int L = slen[b];
+        if (L >= K) {
+            const int32_t *key = stok + (size_t)b * sstride + (L - K);
+            for (int pass = 0; pass < 2 && best_h < 0; ++pass)
+                for (int h = 0; h < H; ++h) {
+                    if (pass == 0 && hgroup[h] != sgroup[b]) continue;
+                    for (int p = 0; p + K < hlen[h]; ++p) {
+                        int eq = 1;
+                        for (int i = 0; i < K && eq; ++i) eq = htok[(size_t)h * hstride + p + i] == key[i];
+                        if (!eq) continue;
+                        if (best_h < 0 || hreward[h] > hreward[best_h]) { best_h = h; best_p = p; }
+                        break;  /* the lowest p of this response */
+                    }
+                }
+        }
+        int n = 0;
+        for (int k = 0; k < gamma; ++k) {
+            int t = 0;
+            if (best_h >= 0 && best_p + K + k < hlen[best_h]) {
+                t = htok[(size_t)best_h * hstride + best_p + K + k];
+                ++n;
+            }
+            drafts[(size_t)b * gamma + k] = t;
+        }
+        draft_len[b] = n;
+        if (probs && vocab > 0)
+            for (int k = 0; k < gamma; ++k) {
+                float *row = probs + ((size_t)b * gamma + k) * vocab;
+                memset(row, 0, sizeof(float) * (size_t)vocab);
+                const int t = drafts[(size_t)b * gamma + k];
+                if (t >= 0 && t < vocab) row[t] = 1.f;
+            }
+    }
+    return 0;
+}
