@@ -212,6 +212,45 @@ SV_API sv_status sv_kv_commit(const sv_attn_desc *desc, int32_t num_layers, cons
                               void *stream);
 
 /* ------------------------------------------------------------------------
+ * Weight-free drafts from earlier responses
+ * ------------------------------------------------------------------------
+ * Chain drafts looked up in earlier rollouts' responses instead of drawn from
+ * a draft model (History Tree PR: drafts from earlier high-reward responses of
+ * the same prompt, with a global fallback; SRT review: prefix lookup in
+ * earlier rollouts). For sequence b the key is its last key_len tokens. A
+ * candidate is a response h and position p with history[h][p..p+key_len-1]
+ * equal to the key and at least one token after it; candidates are first
+ * sought among responses of the sequence's group, and among all responses if
+ * none matched. The chosen one has the highest reward, then the lowest h, then
+ * the lowest p. The drafts are the up to gamma tokens after it (draft_len),
+ * padded with token 0; a sequence shorter than key_len or without a candidate
+ * gets draft_len 0. With vocab > 0, draft_probs receives one-hot rows at the
+ * draft tokens (padding included): a draft drawn from that q, as the accept
+ * rule requires. Lengths are clamped to their rows' strides.
+ *   history_tokens int32 [H][history_stride], history_lens [H],
+ *   history_reward fp32 [H], history_group int32 [H]
+ *   seq_tokens int32 [B][seq_stride], seq_lens [B], seq_group [B]
+ *   draft_tokens int32 [B][gamma] out, draft_len int32 [B] out,
+ *   draft_probs fp32 [B][gamma][vocab] out or NULL
+ * Limits: 1 <= key_len <= 64, 1 <= gamma <= 63.
+ */
+typedef struct {
+    int32_t num_seqs;            /* B */
+    int32_t num_history;         /* H */
+    int32_t history_stride;      /* columns of history_tokens */
+    int32_t seq_stride;          /* columns of seq_tokens */
+    int32_t key_len;             /* tokens matched */
+    int32_t gamma;               /* drafts per sequence */
+    int32_t vocab;               /* columns of draft_probs; 0 = no probabilities written */
+} sv_history_desc;
+
+SV_API sv_status sv_history_draft(const sv_history_desc *desc, const int32_t *history_tokens,
+                                  const int32_t *history_lens, const float *history_reward,
+                                  const int32_t *history_group, const int32_t *seq_tokens, const int32_t *seq_lens,
+                                  const int32_t *seq_group, int32_t *draft_tokens, int32_t *draft_len,
+                                  float *draft_probs, void *stream);
+
+/* ------------------------------------------------------------------------
  * Host speculative-decoding controller
  * ------------------------------------------------------------------------
  * Host logic (no GPU work) that decides, for each decode step of a batch,

@@ -17,7 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc", "SvKVLayer",
     "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
-    "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig",
+    "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig", "SvHistoryDesc", "sv_history_draft",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
 ]
@@ -86,6 +86,11 @@ class SvCtlStep(C.Structure):
                 ("accepted_drafts", C.c_int64), ("rejections", C.c_int64), ("step_ms", C.c_double)]
 
 
+class SvHistoryDesc(C.Structure):
+    _fields_ = [("num_seqs", C.c_int32), ("num_history", C.c_int32), ("history_stride", C.c_int32),
+                ("seq_stride", C.c_int32), ("key_len", C.c_int32), ("gamma", C.c_int32), ("vocab", C.c_int32)]
+
+
 class SvAcceptDesc(C.Structure):
     _fields_ = [("num_seqs", C.c_int32), ("num_rows", C.c_int32), ("vocab", C.c_int32),
                 ("tree_parents", C.POINTER(C.c_int32))]
@@ -120,6 +125,8 @@ def _load() -> C.CDLL:
     L.sv_ctl_observe.restype = C.c_int
     L.sv_ctl_acceptance.argtypes = [C.c_void_p]
     L.sv_ctl_acceptance.restype = C.c_double
+    L.sv_history_draft.argtypes = [C.POINTER(SvHistoryDesc)] + [P] * 10 + [P]
+    L.sv_history_draft.restype = C.c_int
     L.sv_status_string.argtypes = [C.c_int]
     L.sv_status_string.restype = C.c_char_p
     L.sv_last_error.argtypes = []
@@ -227,6 +234,14 @@ def sv_kv_commit(desc: SvAttnDesc, layers, block_table, ctx_lens, accept_len, ac
 def make_kv_layers(layers) -> C.Array:
     """The SvKVLayer array of sv_kv_commit, built once for repeated calls."""
     return (SvKVLayer * len(layers))(*[SvKVLayer(_ptr(k), _ptr(v)) for k, v in layers])
+
+
+def sv_history_draft(desc: SvHistoryDesc, history_tokens, history_lens, history_reward, history_group,
+                     seq_tokens, seq_lens, seq_group, draft_tokens, draft_len, draft_probs=None,
+                     stream=None) -> None:
+    _check(_L().sv_history_draft(C.byref(desc), _ptr(history_tokens), _ptr(history_lens), _ptr(history_reward),
+                                 _ptr(history_group), _ptr(seq_tokens), _ptr(seq_lens), _ptr(seq_group),
+                                 _ptr(draft_tokens), _ptr(draft_len), _ptr(draft_probs), _stream(stream)))
 
 
 def default_ctl_config() -> SvCtlConfig:

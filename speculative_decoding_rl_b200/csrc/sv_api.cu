@@ -220,4 +220,36 @@ sv_status sv_kv_commit(const sv_attn_desc *d, int32_t num_layers, const sv_kv_la
     return SV_OK;
 }
 
+sv_status sv_history_draft(const sv_history_desc *d, const int32_t *history_tokens, const int32_t *history_lens,
+                           const float *history_reward, const int32_t *history_group, const int32_t *seq_tokens,
+                           const int32_t *seq_lens, const int32_t *seq_group, int32_t *draft_tokens,
+                           int32_t *draft_len, float *draft_probs, void *stream) {
+    if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
+    if (d->num_seqs < 0 || d->num_history < 0) return fail(SV_ERR_INVALID_ARG, "negative count");
+    if (d->key_len < 1 || d->key_len > 64) return fail(SV_ERR_INVALID_ARG, "key_len must be in [1, 64]");
+    if (d->gamma < 1 || d->gamma > 63) return fail(SV_ERR_INVALID_ARG, "gamma must be in [1, 63]");
+    if (d->history_stride < 1 || d->seq_stride < 1) return fail(SV_ERR_INVALID_ARG, "strides must be positive");
+    if (d->vocab < 0) return fail(SV_ERR_INVALID_ARG, "vocab < 0");
+    if (d->num_seqs == 0) return SV_OK;
+    if (!seq_tokens || !seq_lens || !seq_group || !draft_tokens || !draft_len)
+        return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (d->num_history > 0 && (!history_tokens || !history_lens || !history_reward || !history_group))
+        return fail(SV_ERR_INVALID_ARG, "a history pointer is NULL");
+    if (d->vocab > 0 && !draft_probs) return fail(SV_ERR_INVALID_ARG, "draft_probs is NULL with vocab > 0");
+    const void *ptrs[] = {history_tokens, history_lens, history_reward, history_group, seq_tokens,
+                          seq_lens, seq_group, draft_tokens, draft_len, draft_probs};
+    for (const void *q : ptrs)
+        if (q && !aligned(q, 4)) return fail(SV_ERR_INVALID_ARG, "misaligned pointer");
+    if ((long long)d->num_history * d->history_stride > (1LL << 40)) return fail(SV_ERR_UNSUPPORTED, "history too large");
+    sv::HistoryLaunch h;
+    h.htok = history_tokens; h.hlen = history_lens; h.hgroup = history_group; h.hreward = history_reward;
+    h.stok = seq_tokens; h.slen = seq_lens; h.sgroup = seq_group;
+    h.drafts = draft_tokens; h.dlen = draft_len; h.probs = d->vocab > 0 ? draft_probs : nullptr;
+    h.B = d->num_seqs; h.H = d->num_history; h.hstride = d->history_stride; h.sstride = d->seq_stride;
+    h.K = d->key_len; h.gamma = d->gamma; h.V = d->vocab;
+    cudaError_t e = sv::launch_history_draft(h, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SV_ERR_CUDA, "history draft launch: %s", cudaGetErrorString(e));
+    return SV_OK;
+}
+
 }  // extern "C"

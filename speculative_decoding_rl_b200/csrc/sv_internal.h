@@ -72,6 +72,16 @@ struct CommitLaunch {
 };
 cudaError_t launch_kv_commit(const CommitLaunch &c, cudaStream_t stream);
 
+// ---------------------------- history drafts --------------------------------
+struct HistoryLaunch {
+    const int32_t *htok, *hlen, *hgroup, *stok, *slen, *sgroup;
+    const float *hreward;
+    int32_t *drafts, *dlen;
+    float *probs;
+    int B, H, hstride, sstride, K, gamma, V;
+};
+cudaError_t launch_history_draft(const HistoryLaunch &h, cudaStream_t stream);
+
 // Sets the text sv_last_error() returns on the calling thread.
 void record_error(const char *msg);
 

@@ -144,3 +144,24 @@ def test_kv_commit_rejects_null_and_misaligned_pointers():
             sv.sv_kv_commit(d, layers, *args)
         assert e.value.status == 1
     sv.sv_kv_commit(sv.SvAttnDesc(0, 5, 4, 2, 128, 16, 4, 8), [(256, 512)], 0, 0, 0, 0, 0)  # no sequences
+
+
+@pytest.mark.parametrize("kw", [dict(key_len=0), dict(key_len=65), dict(gamma=0), dict(gamma=64),
+                                dict(history_stride=0), dict(vocab=-1), dict(num_seqs=-1)])
+def test_history_draft_rejects_bad_descriptors(kw):
+    base = dict(num_seqs=2, num_history=3, history_stride=16, seq_stride=16, key_len=3, gamma=4, vocab=0)
+    base.update(kw)
+    d = sv.SvHistoryDesc(*[base[k] for k in ("num_seqs", "num_history", "history_stride", "seq_stride",
+                                             "key_len", "gamma", "vocab")])
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_history_draft(d, *([64] * 9))
+    assert e.value.status == 1
+
+
+def test_history_draft_rejects_null_and_misaligned_pointers():
+    d = sv.SvHistoryDesc(2, 3, 16, 16, 3, 4, 8)
+    with pytest.raises(sv.SvError):
+        sv.sv_history_draft(d, 64, 64, 64, 64, 64, 64, 64, 64, 64, None)  # vocab > 0 without probs
+    with pytest.raises(sv.SvError):
+        sv.sv_history_draft(d, 64, 64, 66, 64, 64, 64, 64, 64, 64, 64)
+    sv.sv_history_draft(sv.SvHistoryDesc(0, 3, 16, 16, 3, 4, 0), 0, 0, 0, 0, 0, 0, 0, 0, 0)
