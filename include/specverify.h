@@ -154,7 +154,7 @@ SV_API sv_status sv_verify_attention(const sv_attn_desc *desc, const void *q, co
  * sum_{y<=x} w(y) > u * sum(w), else the last x with w(x) > 0.
  * Arithmetic is fp32. A sequence flagged SV_FLAG_NONFINITE gets
  * accept_len 0, next_token 0; a bad draft token counts as rejected.
- * Limits: 1 <= N <= 64, 1 <= V <= 8*57344, B <= 2^31-1 with grid limits.
+ * Limits: 1 <= N <= 64, 1 <= V <= 450560 (8 x 56320), 0 <= B <= 65535.
  */
 typedef struct {
     int32_t num_seqs;             /* B */
