@@ -150,3 +150,23 @@ def test_split_units_need_no_workspace_initialisation():
     got = first.float().cpu().numpy().astype(np.float64)
     assert_attention_close(got, want, "split units, random workspace")
     assert torch.equal(first, second) and torch.equal(first, third)
+
+
+@pytest.mark.parametrize("name,over,nrows", [
+    ("qwen32b_sweep", dict(num_seqs=64, gamma=8), 64),
+    ("qwen32b_sweep", dict(num_seqs=256, gamma=2), 48),
+    ("grpo_shared_prefix", {}, 64),
+])
+def test_full_size_sampled_rows_other_shapes(name, over, nrows):
+    # the 32B-shaped sweep points (64 and 256 sequences) and the GRPO group with
+    # its shared prompt pages, at full size; the oracle computes sampled rows
+    w = W.workload(name, **over)
+    a = W.build_attention(w)
+    got, st = run(a)
+    assert (st == 0).all()
+    rng = np.random.default_rng(sum(map(ord, name)) + len(over))
+    rows = np.stack([rng.integers(0, a.num_seqs, nrows), rng.integers(0, a.num_q_rows, nrows),
+                     rng.integers(0, a.num_q_heads, nrows)], axis=1).astype(np.int32)
+    want = oracle.attention_rows(a, rows)
+    sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
+    assert_attention_close(sel, want, f"{name} {over} full size, sampled rows")
