@@ -49,6 +49,8 @@ def lib() -> C.CDLL:
         L.orc_attention.restype = i32
         L.orc_attention_rows.argtypes = [i32] * 8 + [P] * 6 + [P, i32, P]
         L.orc_attention_rows.restype = i32
+        L.orc_cascade_attention.argtypes = [i32] * 9 + [P] * 8 + [P, i32, P, P]
+        L.orc_cascade_attention.restype = i32
         L.orc_accept.argtypes = [i32, i32, i32, P, P, P, P, f64, u64, P, P, P, P, P, P, P, P]
         L.orc_accept.restype = i32
         L.orc_inv_cdf.argtypes = [P, i32, f64, P]
@@ -125,6 +127,44 @@ def attention_rows(a, rows: np.ndarray) -> np.ndarray:
     if rc:
         raise ValueError(f"orc_attention_rows returned {rc}")
     return out
+
+
+def cascade_attention(a, group_offsets: Sequence[int], prefix_lens: Sequence[int],
+                      rows: Optional[np.ndarray] = None):
+    """Cascade (shared-prefix) verify attention of an ``AttnInputs``-like object.
+
+    Group g = sequences [group_offsets[g], group_offsets[g+1]); its first
+    prefix_lens[g] keys come from the pages of its first member. Without
+    ``rows``: (fp64 [B][N][Hq][D], flags [B]); with rows (b, i, hq): fp64 [nrows][D].
+    """
+    import torch
+    q = _np(a.q.view(torch.int16), np.uint16)
+    k = _np(a.k_pool.view(torch.int16), np.uint16)
+    v = _np(a.v_pool.view(torch.int16), np.uint16)
+    tbl = _np(a.block_table, np.int32)
+    lens = _np(a.ctx_lens, np.int32)
+    mask = _np(a.draft_mask, np.uint64) if a.draft_mask is not None else None
+    off = np.ascontiguousarray(group_offsets, dtype=np.int32)
+    pre = np.ascontiguousarray(prefix_lens, dtype=np.int32)
+    G = len(pre)
+    if off.shape[0] != G + 1:
+        raise ValueError("group_offsets needs one entry more than prefix_lens")
+    if rows is None:
+        out = np.zeros((a.num_seqs, a.num_q_rows, a.num_q_heads, a.head_dim), dtype=np.float64)
+        flags = np.zeros(a.num_seqs, dtype=np.int32)
+        r, nr = None, 0
+    else:
+        r = np.ascontiguousarray(rows, dtype=np.int32).reshape(-1, 3)
+        nr = r.shape[0]
+        out = np.zeros((nr, a.head_dim), dtype=np.float64)
+        flags = None
+    rc = lib().orc_cascade_attention(a.num_seqs, a.num_q_rows, a.num_q_heads, a.num_kv_heads,
+                                     a.head_dim, a.block_size, a.max_blocks_per_seq, a.num_blocks,
+                                     G, _p(off), _p(pre), _p(q), _p(k), _p(v), _p(tbl), _p(lens),
+                                     _p(mask), _p(r), nr, _p(out), _p(flags))
+    if rc:
+        raise ValueError(f"orc_cascade_attention returned {rc}")
+    return out if rows is not None else (out, flags)
 
 
 class AcceptResult:

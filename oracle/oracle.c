@@ -16,6 +16,10 @@
  *    when no mask is given). Scores are q.k/sqrt(D) and the output is the
  *    softmax-weighted sum of V. GQA: query head hq reads KV head hq/(Hq/Hkv).
  *
+ *  - Cascade verify attention: the same attention for groups of rollouts
+ *    that share a prompt's KV pages (SRT review, "Tree-Structured KV
+ *    Cache"): the group's prefix keys come from one set of pages.
+ *
  *  - Accept / resample: the lossless rule (Accelerating RL Post-Training
  *    Rollouts via System-Integrated Speculative Decoding, Abstract: speculative
  *    decoding preserves the target's output distribution), with drafts after
@@ -206,6 +210,83 @@ int orc_attention_rows(int B, int N, int Hq, int Hkv, int D, int bs, int max_blo
         else
             for (int d = 0; d < D; ++d) o[d] = 0.0;
     }
+    free(scratch);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Cascade (shared-prefix) verify attention                                  */
+/* ------------------------------------------------------------------------ */
+
+/* Rollouts of one prompt share its KV pages: a shared prefix node is stored
+ * once and every rollout that passes through it reads it (SRT review, "Core
+ * idea" and "Tree-Structured KV Cache", node sharing). The operation is plain
+ * verify attention over each member's whole context, where the first
+ * prefix_lens[g] keys of every member of group g come from the pages of the
+ * group's first member and the rest from the member's own block table row.
+ *
+ * Groups are consecutive: group g holds sequences [off[g], off[g+1]), with
+ * off[0] = 0, off[G] = B, nondecreasing. A member is valid when prefix_lens[g]
+ * is a non-negative multiple of bs, prefix_lens[g] <= ctx_len - N, and its
+ * effective table row passes seq_valid. An invalid member gets zeros and flag 1.
+ *
+ * rows == NULL: out is fp64 [B][N][Hq][D] and flags [B] (may be NULL).
+ * rows != NULL: rows[3r..3r+2] = (b, i, hq); out is fp64 [nrows][D]. */
+int orc_cascade_attention(int B, int N, int Hq, int Hkv, int D, int bs, int max_blocks,
+                          int num_blocks, int num_groups, const int32_t *group_offsets,
+                          const int32_t *prefix_lens, const uint16_t *q, const uint16_t *k_pool,
+                          const uint16_t *v_pool, const int32_t *block_table,
+                          const int32_t *ctx_lens, const uint64_t *mask, const int32_t *rows,
+                          int nrows, double *out, int32_t *flags)
+{
+    if (B < 0 || N < 1 || N > 64 || Hq < 1 || Hkv < 1 || Hq % Hkv || D < 1 || bs < 1) return -2;
+    if (num_groups < 0 || group_offsets[0] != 0 || group_offsets[num_groups] != B) return -2;
+    for (int g = 0; g < num_groups; ++g)
+        if (group_offsets[g + 1] < group_offsets[g]) return -2;
+    int32_t *eff = (int32_t *)malloc(sizeof(int32_t) * ((size_t)B * max_blocks + 1));
+    int *ok = (int *)malloc(sizeof(int) * ((size_t)B + 1));
+    int cmax = 1;
+    for (int b = 0; b < B; ++b) if (ctx_lens[b] > cmax) cmax = ctx_lens[b];
+    double *scratch = (double *)malloc(sizeof(double) * (size_t)cmax);
+    if (!eff || !ok || !scratch) { free(eff); free(ok); free(scratch); return -3; }
+    /* each member's effective page list: the group's prefix pages, then its own */
+    for (int g = 0; g < num_groups; ++g) {
+        const int first = group_offsets[g], P = prefix_lens[g];
+        for (int b = group_offsets[g]; b < group_offsets[g + 1]; ++b) {
+            const int pre_ok = P >= 0 && P % bs == 0 && P <= ctx_lens[b] - N;
+            for (int j = 0; j < max_blocks; ++j) {
+                const int from = (pre_ok && j < P / bs) ? first : b;
+                eff[(size_t)b * max_blocks + j] = block_table[(size_t)from * max_blocks + j];
+            }
+            ok[b] = pre_ok && seq_valid(N, bs, max_blocks, num_blocks, eff, ctx_lens, b);
+        }
+    }
+    if (!rows) {
+        for (int b = 0; b < B; ++b) {
+            for (int i = 0; i < N; ++i)
+                for (int hq = 0; hq < Hq; ++hq) {
+                    double *o = out + (((size_t)b * N + i) * Hq + hq) * D;
+                    if (ok[b])
+                        attention_row(N, Hq, Hkv, D, bs, max_blocks, q, k_pool, v_pool, eff,
+                                      ctx_lens, mask, b, i, hq, o, scratch);
+                    else
+                        for (int d = 0; d < D; ++d) o[d] = 0.0;
+                }
+            if (flags) flags[b] = !ok[b];
+        }
+    } else {
+        for (int r = 0; r < nrows; ++r) {
+            const int b = rows[3 * r], i = rows[3 * r + 1], hq = rows[3 * r + 2];
+            double *o = out + (size_t)r * D;
+            if (ok[b])
+                attention_row(N, Hq, Hkv, D, bs, max_blocks, q, k_pool, v_pool, eff, ctx_lens,
+                              mask, b, i, hq, o, scratch);
+            else
+                for (int d = 0; d < D; ++d) o[d] = 0.0;
+        }
+    }
+    free(eff);
+    free(ok);
     free(scratch);
     return 0;
 }

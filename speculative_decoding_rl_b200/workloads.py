@@ -84,6 +84,10 @@ class AttnInputs:
     ctx_lens: torch.Tensor     # int32 [B] (includes the N new positions)
     draft_mask: Optional[torch.Tensor]  # int64 view of uint64 [B][N], or None for a chain
     guard_block: int
+    # groups of consecutive sequences sharing prefix pages (None: no groups):
+    # group g = sequences [group_offsets[g], group_offsets[g+1]), prefix_lens[g] shared keys
+    group_offsets: Optional[List[int]] = None
+    prefix_lens: Optional[List[int]] = None
 
     def kv_bytes_unique(self) -> int:
         """Bytes of K and V pages that hold at least one visible key (shared pages once)."""
@@ -224,10 +228,14 @@ def make_attention_inputs(num_q_rows: int, num_q_heads: int, num_kv_heads: int, 
         m = ancestor_masks(par)
         mask = torch.from_numpy(np.tile(m, (B, 1)).view(np.int64).copy())
 
+    offsets = prefix = None
+    if shared_prefix_groups:
+        offsets = [g * group_size for g in range(shared_prefix_groups + 1)]
+        prefix = [int(shared_prefix_tokens)] * shared_prefix_groups
     return AttnInputs(B, N, num_q_heads, num_kv_heads, head_dim, bs, mb, num_blocks,
                       q.contiguous(), k_pool.contiguous(), v_pool.contiguous(),
                       torch.from_numpy(table), torch.tensor(list(ctx_lens), dtype=torch.int32),
-                      mask, guard)
+                      mask, guard, offsets, prefix)
 
 
 def make_accept_inputs(num_seqs: int, num_rows: int, vocab: int, seed: int, *,
