@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
     ap.add_argument("--num-seqs", type=int, default=None, help="active sequences B (qwen32b_sweep)")
     ap.add_argument("--gamma", type=int, default=None, help="chain drafts per sequence (qwen32b_sweep)")
+    ap.add_argument("--cascade", action="store_true",
+                    help="read each group's shared prompt pages once (sv_cascade_verify_attention); "
+                         "workloads whose sequences come in groups only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
@@ -263,7 +266,7 @@ def run_reference(args, world, rank):
 
 def run_ours(args, world, rank, local):
     import speculative_decoding_rl_b200 as sv
-    from speculative_decoding_rl_b200.session import AcceptCall, AttentionCall
+    from speculative_decoding_rl_b200.session import AcceptCall, AttentionCall, CascadeCall
 
     dev = torch.device("cuda", local)
     w = make_workload(args)
@@ -271,19 +274,24 @@ def run_ours(args, world, rank, local):
     a0 = W.build_attention(w)
     acc_in = W.build_accept(w)
     B, N, Hq, D = a0.num_seqs, a0.num_q_rows, a0.num_q_heads, a0.head_dim
+    if args.cascade and a0.group_offsets is None:
+        raise SystemExit(f"--cascade: workload {w.name} has no groups of sequences sharing a prefix")
+    Call = CascadeCall if args.cascade else AttentionCall
 
     # Layer 0 from the seeded CPU generator; layers 1.. get their own pools and
     # queries drawn on the device (same sequences and page tables). Distinct pools
     # are capped by POOL_BUDGET_BYTES; past that, layers reuse pools cyclically.
-    calls = [AttentionCall(a0, device=str(dev))]
+    calls = [Call(a0, device=str(dev))]
     g = torch.Generator(device=dev)
     g.manual_seed(1234 + rank)
     pool_bytes = 2 * a0.k_pool.numel() * 2
     n_pools = max(1, min(layers, POOL_BUDGET_BYTES // max(1, pool_bytes)))
     for li in range(1, layers):
-        c = AttentionCall.__new__(AttentionCall)
+        c = Call.__new__(Call)
         c.inputs = a0
         c.desc = calls[0].desc
+        if args.cascade:
+            c.cdesc = calls[0].cdesc
         c.block_table, c.ctx_lens, c.mask = calls[0].block_table, calls[0].ctx_lens, calls[0].mask
         if li < n_pools:
             c.k_pool = torch.randn(a0.k_pool.shape, generator=g, device=dev, dtype=torch.bfloat16)
@@ -318,7 +326,8 @@ def run_ours(args, world, rank, local):
     step(0)
     torch.cuda.synchronize()
     rows = np.stack([np.arange(16) % B, (np.arange(16) * 3) % N, (np.arange(16) * 7) % Hq], 1).astype(np.int32)
-    ref = oracle.attention_rows(a0, rows)
+    ref = (oracle.cascade_attention(a0, a0.group_offsets, a0.prefix_lens, rows=rows) if args.cascade
+           else oracle.attention_rows(a0, rows))
     got = calls[0].out.float().cpu().numpy()[rows[:, 0], rows[:, 1], rows[:, 2]]
     parity_attn = float(np.abs(got - ref).max())
     o = oracle.accept(acc_in.target_logits, acc_in.draft_probs, acc_in.draft_tokens, acc_in.temperature, 0,
@@ -356,6 +365,21 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     call_times = [a.elapsed_time(b) / 1e3 for pairs in ev_all for a, b in pairs]
     t_attn = float(np.mean(call_times))
+    t_plain = None
+    if args.cascade:
+        # the plain call on the same inputs (its workspace is the front of the cascade's)
+        ev_plain = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)]
+                    for _ in range(min(K, 5) * layers)]
+        for c in calls:
+            AttentionCall.run(c, stream)
+        for r in range(min(K, 5)):
+            for li, c in enumerate(calls):
+                e0, e1 = ev_plain[r * layers + li]
+                e0.record(stream)
+                AttentionCall.run(c, stream)
+                e1.record(stream)
+        torch.cuda.synchronize()
+        t_plain = float(np.mean([a.elapsed_time(b) / 1e3 for a, b in ev_plain]))
 
     elapsed_max = max_over_ranks(elapsed, world)
     steps_total = sum_over_ranks(float(K), world)
@@ -478,18 +502,21 @@ def run_ours(args, world, rank, local):
             "config": {"workload": w.name, "layers": layers, "num_seqs": B, "gamma": N - 1,
                        "q_heads": Hq, "kv_heads": a0.num_kv_heads, "head_dim": D,
                        "ctx_tokens_total": int(a0.ctx_lens.sum()), "vocab": acc_in.vocab,
-                       "temperature": acc_in.temperature,
+                       "temperature": acc_in.temperature, "cascade": bool(args.cascade),
                        "l2": ("inputs larger than L2 (every layer has its own KV pool)" if n_pools == layers else
                               f"inputs larger than L2 ({n_pools} KV pools of {pool_bytes / 1e9:.1f} GB cycled over {layers} layers)"),
                        "parallelism": f"replicas x{world}"},
             "accepted_tok_s": tok_s,
             "t_attn_call_ms": 1e3 * t_attn, "t_accept_call_ms": 1e3 * t_acc,
+            "t_attn_plain_call_ms": None if t_plain is None else 1e3 * t_plain,
             "hbm_gbs_step": step_bytes / (elapsed_max / K) / 1e9,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": recorded_traffic(w.name),
-                         "kernel": "sv_verify_attention call: attn_tc_kernel + attn_combine_kernel",
+                         "frac": achieved / peak, "traffic": None if args.cascade else recorded_traffic(w.name),
+                         "kernel": ("sv_cascade_verify_attention call: cascade_prep_kernel + cascade_prefix_kernel"
+                                    " + attn_tc_kernel + attn_combine_kernel" if args.cascade else
+                                    "sv_verify_attention call: attn_tc_kernel + attn_combine_kernel"),
                          "algorithmic_bytes_per_call": alg_bytes, "peak_source": peak_kind},
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * (2 * layers + 1),
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": K * ((4 if args.cascade else 2) * layers + 1),
             "clocks": clocks, "parity": parity, "kv_commit": commit_info,
         }
         print(json.dumps(line), flush=True)

@@ -123,6 +123,53 @@ SV_API sv_status sv_verify_attention(const sv_attn_desc *desc, const void *q, co
                               size_t workspace_bytes, int32_t *status_flags, void *stream);
 
 /* ------------------------------------------------------------------------
+ * Cascade verify attention (rollout groups that share a prompt's KV pages)
+ * ------------------------------------------------------------------------
+ * The rollouts of one prompt share its prefix, whose KV is stored once and
+ * read by every rollout that passes through it (SRT review, "Core idea" and
+ * "Tree-Structured KV Cache": node sharing; "Speculative Rollout
+ * integration": shared-prefix KV reuse and fewer memory accesses as the
+ * speed-up sources). This call returns what sv_verify_attention returns for
+ * each member's whole context, except that the first prefix_lens[g] keys of
+ * every member of group g are read from the pages of the group's FIRST member
+ * (block_table row group_offsets[g]); the other members' first
+ * prefix_lens[g]/16 table entries are not read. Those shared keys are read once
+ * per group and KV head for all the group's query rows (a tensor-core pass over
+ * the group's rows), the members' own keys by the split-context pass of
+ * sv_verify_attention, and the two partial softmaxes are merged by log-sum-exp.
+ *
+ * cdesc and both of its arrays are HOST memory, read during the call:
+ *   num_groups      1 .. SV_CASCADE_MAX_GROUPS
+ *   group_offsets   int32 [num_groups + 1]: group g is sequences
+ *                   [group_offsets[g], group_offsets[g+1]); group_offsets[0] = 0,
+ *                   group_offsets[num_groups] = num_seqs, nondecreasing
+ *   prefix_lens     int32 [num_groups]: shared keys of each group, a multiple
+ *                   of 16 in [0, max_blocks_per_seq * 16]
+ * Every other argument, limit and error as sv_verify_attention, with the
+ * workspace size from sv_cascade_attention_workspace_size. On the device, a
+ * member whose context is invalid or shorter than prefix_lens[g] + N gets
+ * SV_FLAG_BAD_CONTEXT and out = 0; a block id outside the pool among the
+ * group's prefix pages gives every member SV_FLAG_BAD_BLOCK (zeros are read
+ * for that page).
+ */
+#define SV_CASCADE_MAX_GROUPS 128
+typedef struct {
+    int32_t num_groups;
+    const int32_t *group_offsets;  /* HOST [num_groups + 1] */
+    const int32_t *prefix_lens;    /* HOST [num_groups] */
+} sv_cascade_desc;
+
+/* Bytes of device workspace sv_cascade_verify_attention needs; 0 on an invalid
+ * desc or cdesc. */
+SV_API size_t sv_cascade_attention_workspace_size(const sv_attn_desc *desc, const sv_cascade_desc *cdesc);
+
+SV_API sv_status sv_cascade_verify_attention(const sv_attn_desc *desc, const sv_cascade_desc *cdesc,
+                                             const void *q, const sv_paged_kv *paged_kv,
+                                             const int32_t *block_table, const int32_t *ctx_lens,
+                                             const uint64_t *draft_mask, void *out, void *workspace,
+                                             size_t workspace_bytes, int32_t *status_flags, void *stream);
+
+/* ------------------------------------------------------------------------
  * Accept / resample
  * ------------------------------------------------------------------------
  * Shapes:

@@ -17,6 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc", "SvKVLayer",
     "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
+    "SvCascadeDesc", "make_cascade_desc", "sv_cascade_attention_workspace_size", "sv_cascade_verify_attention",
     "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig", "SvHistoryDesc", "sv_history_draft",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
@@ -37,6 +38,7 @@ SV_CTL_GAMMA_ACCEPTANCE, SV_CTL_GAMMA_MAB = 0, 1
 SV_DRAFTER_NONE, SV_DRAFTER_HISTORY, SV_DRAFTER_MODEL = 0, 1, 2
 SV_CTL_MAX_BUCKETS = 64
 SV_NOALLOC_SCRATCH_BYTES = 64 << 20
+SV_CASCADE_MAX_GROUPS = 128
 
 
 class SvError(RuntimeError):
@@ -53,6 +55,11 @@ class SvAttnDesc(C.Structure):
 
 class SvPagedKV(C.Structure):
     _fields_ = [("k_pool", C.c_void_p), ("v_pool", C.c_void_p)]
+
+
+class SvCascadeDesc(C.Structure):
+    _fields_ = [("num_groups", C.c_int32), ("group_offsets", C.POINTER(C.c_int32)),
+                ("prefix_lens", C.POINTER(C.c_int32))]
 
 
 class SvKVLayer(C.Structure):
@@ -109,6 +116,11 @@ def _load() -> C.CDLL:
     L.sv_verify_attention.restype = C.c_int
     L.sv_verify_attention_noalloc.argtypes = [C.POINTER(SvAttnDesc), P, C.POINTER(SvPagedKV), P, P, P, P, P, P]
     L.sv_verify_attention_noalloc.restype = C.c_int
+    L.sv_cascade_attention_workspace_size.argtypes = [C.POINTER(SvAttnDesc), C.POINTER(SvCascadeDesc)]
+    L.sv_cascade_attention_workspace_size.restype = sz
+    L.sv_cascade_verify_attention.argtypes = [C.POINTER(SvAttnDesc), C.POINTER(SvCascadeDesc), P,
+                                              C.POINTER(SvPagedKV), P, P, P, P, P, sz, P, P]
+    L.sv_cascade_verify_attention.restype = C.c_int
     L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P]
     L.sv_accept.restype = C.c_int
     L.sv_kv_commit.argtypes = [C.POINTER(SvAttnDesc), i32, C.POINTER(SvKVLayer), P, P, P, P, P, P, P]
@@ -211,6 +223,33 @@ def sv_verify_attention_noalloc(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_
     array (SV_NOALLOC_SCRATCH_BYTES). Calls that overlap on the GPU race on it."""
     _check(_L().sv_verify_attention_noalloc(C.byref(desc), _ptr(q), C.byref(paged_kv), _ptr(block_table),
                                             _ptr(ctx_lens), _ptr(draft_mask), _ptr(out), _ptr(status_flags),
+                                            _stream(stream)))
+
+
+def make_cascade_desc(group_offsets: Sequence[int], prefix_lens: Sequence[int]) -> SvCascadeDesc:
+    """The host-side group description of sv_cascade_verify_attention; it keeps its arrays alive."""
+    n = len(prefix_lens)
+    off = (C.c_int32 * (n + 1))(*[int(x) for x in group_offsets])
+    pre = (C.c_int32 * max(n, 1))(*[int(x) for x in prefix_lens])
+    if len(group_offsets) != n + 1:
+        raise ValueError("group_offsets needs one entry more than prefix_lens")
+    d = SvCascadeDesc(n, C.cast(off, C.POINTER(C.c_int32)), C.cast(pre, C.POINTER(C.c_int32)))
+    d._keep = (off, pre)
+    return d
+
+
+def sv_cascade_attention_workspace_size(desc: SvAttnDesc, cdesc: SvCascadeDesc) -> int:
+    return int(_L().sv_cascade_attention_workspace_size(C.byref(desc), C.byref(cdesc)))
+
+
+def sv_cascade_verify_attention(desc: SvAttnDesc, cdesc: SvCascadeDesc, q, paged_kv: SvPagedKV, block_table,
+                                ctx_lens, draft_mask, out, workspace, workspace_bytes: int, status_flags=None,
+                                stream=None) -> None:
+    """sv_verify_attention for groups of consecutive sequences that share their first
+    prefix_lens[g] keys on the pages of the group's first member."""
+    _check(_L().sv_cascade_verify_attention(C.byref(desc), C.byref(cdesc), _ptr(q), C.byref(paged_kv),
+                                            _ptr(block_table), _ptr(ctx_lens), _ptr(draft_mask), _ptr(out),
+                                            _ptr(workspace), int(workspace_bytes), _ptr(status_flags),
                                             _stream(stream)))
 
 

@@ -42,6 +42,67 @@ sv_status check_attn_desc(const sv_attn_desc *d) {
     return SV_OK;
 }
 
+sv_status check_cascade_desc(const sv_attn_desc *d, const sv_cascade_desc *c) {
+    if (!c) return fail(SV_ERR_INVALID_ARG, "cascade desc is NULL");
+    if (c->num_groups < 1 || c->num_groups > SV_CASCADE_MAX_GROUPS)
+        return fail(SV_ERR_INVALID_ARG, "num_groups must be in [1, %d]", SV_CASCADE_MAX_GROUPS);
+    if (!c->group_offsets || !c->prefix_lens) return fail(SV_ERR_INVALID_ARG, "group_offsets or prefix_lens is NULL");
+    if (c->group_offsets[0] != 0 || c->group_offsets[c->num_groups] != d->num_seqs)
+        return fail(SV_ERR_INVALID_ARG, "group_offsets must run from 0 to num_seqs");
+    for (int g = 0; g < c->num_groups; ++g) {
+        if (c->group_offsets[g + 1] < c->group_offsets[g])
+            return fail(SV_ERR_INVALID_ARG, "group_offsets must be nondecreasing");
+        const int P = c->prefix_lens[g];
+        if (P < 0 || P % sv::PAGE || (long long)P > (long long)d->max_blocks_per_seq * sv::PAGE)
+            return fail(SV_ERR_INVALID_ARG, "prefix_lens[%d] must be a multiple of 16 in [0, max_blocks_per_seq*16]", g);
+    }
+    return SV_OK;
+}
+
+// Pointer checks shared by the plain and the cascade call.
+sv_status check_attn_ptrs(const void *q, const sv_paged_kv *kv, const int32_t *block_table,
+                          const int32_t *ctx_lens, const uint64_t *draft_mask, const void *out,
+                          const int32_t *status_flags) {
+    if (!q || !kv || !kv->k_pool || !kv->v_pool || !block_table || !ctx_lens || !out)
+        return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(kv->k_pool, 16) || !aligned(kv->v_pool, 16))
+        return fail(SV_ERR_INVALID_ARG, "q, out and the KV pools must be 16-byte aligned");
+    if (!aligned(block_table, 4) || !aligned(ctx_lens, 4) || (status_flags && !aligned(status_flags, 4)) ||
+        (draft_mask && !aligned(draft_mask, 8)))
+        return fail(SV_ERR_INVALID_ARG, "misaligned table, length, mask or status pointer");
+    return SV_OK;
+}
+
+sv::AttnParams attn_params(const sv_attn_desc *d, const void *q, const sv_paged_kv *kv,
+                           const int32_t *block_table, const int32_t *ctx_lens, const uint64_t *draft_mask,
+                           void *out, void *workspace, int32_t *status_flags, int ctas) {
+    sv::AttnParams p = {};
+    p.q = static_cast<const uint16_t *>(q);
+    p.k_pool = static_cast<const uint16_t *>(kv->k_pool);
+    p.v_pool = static_cast<const uint16_t *>(kv->v_pool);
+    p.block_table = block_table;
+    p.ctx_lens = ctx_lens;
+    p.mask = draft_mask;
+    p.out = static_cast<uint16_t *>(out);
+    p.status = status_flags;
+    p.B = d->num_seqs;
+    p.N = d->num_q_rows;
+    p.Hq = d->num_q_heads;
+    p.Hkv = d->num_kv_heads;
+    p.D = d->head_dim;
+    p.G = p.Hq / p.Hkv;
+    p.R = p.N * p.G;
+    int nc = 0;
+    sv::row_chunks(p.N, p.G, &p.rows_unit, &p.RC, &nc);
+    p.max_blocks = d->max_blocks_per_seq;
+    p.num_blocks = d->num_blocks;
+    p.units = p.B * p.Hkv * p.RC;
+    p.num_ctas = ctas;
+    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
+    p.ws_partial = static_cast<float *>(workspace);
+    return p;
+}
+
 }  // namespace
 
 namespace sv {
@@ -80,13 +141,7 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
     sv_status s = check_attn_desc(d);
     if (s != SV_OK) return s;
     if (d->num_seqs == 0) return SV_OK;
-    if (!q || !kv || !kv->k_pool || !kv->v_pool || !block_table || !ctx_lens || !out)
-        return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
-    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(kv->k_pool, 16) || !aligned(kv->v_pool, 16))
-        return fail(SV_ERR_INVALID_ARG, "q, out and the KV pools must be 16-byte aligned");
-    if (!aligned(block_table, 4) || !aligned(ctx_lens, 4) || (status_flags && !aligned(status_flags, 4)) ||
-        (draft_mask && !aligned(draft_mask, 8)))
-        return fail(SV_ERR_INVALID_ARG, "misaligned table, length, mask or status pointer");
+    if ((s = check_attn_ptrs(q, kv, block_table, ctx_lens, draft_mask, out, status_flags)) != SV_OK) return s;
     const int ctas = sv::attention_num_ctas();
     if (ctas <= 0) return fail(SV_ERR_CUDA, "cannot query the current device");
     const size_t need = sv::attention_workspace_bytes(d->num_seqs, d->num_q_rows, d->num_q_heads,
@@ -94,32 +149,47 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
         return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);
 
-    sv::AttnParams p = {};
-    p.q = static_cast<const uint16_t *>(q);
-    p.k_pool = static_cast<const uint16_t *>(kv->k_pool);
-    p.v_pool = static_cast<const uint16_t *>(kv->v_pool);
-    p.block_table = block_table;
-    p.ctx_lens = ctx_lens;
-    p.mask = draft_mask;
-    p.out = static_cast<uint16_t *>(out);
-    p.status = status_flags;
-    p.B = d->num_seqs;
-    p.N = d->num_q_rows;
-    p.Hq = d->num_q_heads;
-    p.Hkv = d->num_kv_heads;
-    p.D = d->head_dim;
-    p.G = p.Hq / p.Hkv;
-    p.R = p.N * p.G;
-    int nc = 0;
-    sv::row_chunks(p.N, p.G, &p.rows_unit, &p.RC, &nc);
-    p.max_blocks = d->max_blocks_per_seq;
-    p.num_blocks = d->num_blocks;
-    p.units = p.B * p.Hkv * p.RC;
-    p.num_ctas = ctas;
-    p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
-    p.ws_partial = static_cast<float *>(workspace);
+    const sv::AttnParams p =
+        attn_params(d, q, kv, block_table, ctx_lens, draft_mask, out, workspace, status_flags, ctas);
     cudaError_t e = sv::launch_attention(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(SV_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+    return SV_OK;
+}
+
+size_t sv_cascade_attention_workspace_size(const sv_attn_desc *d, const sv_cascade_desc *c) {
+    if (check_attn_desc(d) != SV_OK || check_cascade_desc(d, c) != SV_OK) return 0;
+    const int ctas = sv::attention_num_ctas();
+    if (ctas <= 0) return 0;
+    sv::CascadePlan plan;
+    sv::cascade_plan(c, d->num_q_rows, d->num_q_heads, d->num_kv_heads, ctas, &plan);
+    return sv::cascade_workspace(d->num_seqs, d->num_q_rows, d->num_q_heads, d->num_kv_heads, d->head_dim,
+                                 d->max_blocks_per_seq, ctas, plan.splits)
+        .total;
+}
+
+sv_status sv_cascade_verify_attention(const sv_attn_desc *d, const sv_cascade_desc *c, const void *q,
+                                      const sv_paged_kv *kv, const int32_t *block_table,
+                                      const int32_t *ctx_lens, const uint64_t *draft_mask, void *out,
+                                      void *workspace, size_t workspace_bytes, int32_t *status_flags,
+                                      void *stream) {
+    sv_status s = check_attn_desc(d);
+    if (s != SV_OK) return s;
+    if ((s = check_cascade_desc(d, c)) != SV_OK) return s;
+    if (d->num_seqs == 0) return SV_OK;
+    if ((s = check_attn_ptrs(q, kv, block_table, ctx_lens, draft_mask, out, status_flags)) != SV_OK) return s;
+    const int ctas = sv::attention_num_ctas();
+    if (ctas <= 0) return fail(SV_ERR_CUDA, "cannot query the current device");
+    sv::CascadePlan plan;
+    sv::cascade_plan(c, d->num_q_rows, d->num_q_heads, d->num_kv_heads, ctas, &plan);
+    const size_t need = sv::cascade_workspace(d->num_seqs, d->num_q_rows, d->num_q_heads, d->num_kv_heads,
+                                              d->head_dim, d->max_blocks_per_seq, ctas, plan.splits)
+                            .total;
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);
+    const sv::AttnParams p =
+        attn_params(d, q, kv, block_table, ctx_lens, draft_mask, out, workspace, status_flags, ctas);
+    cudaError_t e = sv::launch_cascade(p, plan, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(SV_ERR_CUDA, "cascade attention launch: %s", cudaGetErrorString(e));
     return SV_OK;
 }
 

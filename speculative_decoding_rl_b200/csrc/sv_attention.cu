@@ -555,6 +555,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const int tpre = ups * TP[fb] + fhr * Tb;
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
+            // a cascade call merges every unit with its shared prefix: always a slot
+            const bool to_slot = nseg > 1 || p.pp_o != nullptr;
             float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
             // O^T in chunks of 16 columns (few live registers)
 #pragma unroll 1
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 tmem_ld16(lane_base + (2 + pend_ob) * RPa + col0 + c0, o);
                 tmem_wait_ld();
                 if (ell >= D) continue;
-                if (nseg == 1) {
+                if (!to_slot) {
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int r = col0 + c0 + c;
@@ -583,7 +585,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             }
             tc_fence_before();
             warp_arrive(&o_free[pend_ob]);
-            if (nseg > 1 && wiw == 0 && lane < CW && col0 + lane < frows) {
+            if (to_slot && wiw == 0 && lane < CW && col0 + lane < frows) {
                 slot[(size_t)p.rows_unit * D + col0 + lane] = mfin[col0 + lane];
                 slot[(size_t)p.rows_unit * D + p.rows_unit + col0 + lane] = lfin[col0 + lane];
             }
@@ -801,6 +803,8 @@ SV_DEV int block_sum_i(int v, int *red) {
 // sequence by its status warp). One CTA per (COMBINE_ROWS rows, unit), one warp
 // per row, four head dimensions per lane:
 //   M = max_k m_k,  L = sum_k 2^(m_k - M) l_k,  out = sum_k 2^(m_k - M) O_k / L.
+// In a cascade call every unit has slots and the shared prefix's partials of
+// the row join the merge as further terms k.
 // Launched as a programmatic dependent of the attention kernel, which lets it
 // launch only after its own wait on earlier work: the schedule is recomputed
 // from ctx_lens (complete by then) before this kernel waits, so once the
@@ -826,12 +830,17 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     tot = block_sum_i(tot, red_i);
     before = block_sum_i(before, red_i);
     const int Tb = block_sum_i(own, red_i);
+    if (p.pp_o && p.status && blockIdx.x == 0 && hr == 0 && threadIdx.x == 0) {
+        griddep_wait();  // after the attention kernel's status store
+        const int f = __ldcg(p.pflag + b);
+        if (f) atomicOr(p.status + b, f);
+    }
     if (Tb == 0 || r >= rows) return;
     const int total = ups * tot;
     const int W = (total + p.num_ctas - 1) / p.num_ctas;
     const int tpre = ups * before + hr * Tb;
     const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
-    if (n == 1) return;
+    if (n == 1 && !p.pp_o) return;
     const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const size_t sf = slot_stride(RU, D);
@@ -853,6 +862,9 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     float M = mk;
     for (int k = lane + 32; k < n; k += 32) M = fmaxf(M, __ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r));
     M = warp_max(M);
+    const int S = p.pp_o ? p.pp_splits : 0;  // shared-prefix partials of this row
+    const size_t prow = ((size_t)b * p.N + i) * p.Hq + hq, pstride = (size_t)p.B * p.N * p.Hq;
+    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p.pp_ml + 2 * (s * pstride + prow)));
     const float wl = lane < n ? exp2f(mk - M) : 0.f;  // an empty segment holds l = 0
     float L = wl * lk;
     for (int k = lane + 32; k < n; k += 32) {
@@ -861,6 +873,16 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     }
     L = warp_sum(L);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < S; ++s) {
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.pp_ml) + s * pstride + prow);
+        const float w = exp2f(ml.x - M);
+        L = fmaf(w, ml.y, L);
+        if (dl) {
+            const float4 o = __ldcg(reinterpret_cast<const float4 *>(p.pp_o + (s * pstride + prow) * D) + lane);
+            acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
+        }
+    }
 #pragma unroll
     for (int k = 0; k < COMBINE_REG_SEGS; ++k) {
         const float w = __shfl_sync(0xffffffffu, wl, k);

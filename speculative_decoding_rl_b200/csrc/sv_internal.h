@@ -54,6 +54,13 @@ struct AttnParams {
     int units;                 // B * Hkv * RC
     int num_ctas;
     float scale_log2;          // log2(e) / sqrt(D)
+    // Cascade call (null pp_o: a plain call). Every unit then leaves a slot,
+    // and the combine kernel folds in pp_splits partials of the shared prefix
+    // per row and ORs pflag into the status.
+    const float *pp_o;         // [pp_splits][B][N][Hq][D] unnormalised O
+    const float *pp_ml;        // [pp_splits][B][N][Hq][2] running max (log2 domain), row sum
+    const int32_t *pflag;      // [B] status bits found on the prefix pages
+    int pp_splits;
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
@@ -61,6 +68,32 @@ size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_c
 void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc);
 int attention_num_ctas();
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
+
+// ------------------------------ cascade ------------------------------------
+// Shared-prefix pass: one CTA of CASCADE_ROWS query rows per (group, KV head,
+// row chunk, prefix split).
+constexpr int CASCADE_ROWS = 64;
+constexpr int CASCADE_KEYS = 64;
+
+struct CascadePlan {
+    int num_groups, splits, items;
+    int off[SV_CASCADE_MAX_GROUPS + 1];    // group member offsets
+    int pre[SV_CASCADE_MAX_GROUPS];        // shared keys per group
+    int item0[SV_CASCADE_MAX_GROUPS + 1];  // first work item of each group
+};
+
+// Work items and prefix splits for a validated cascade descriptor.
+void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, int num_sms, CascadePlan *plan);
+// Workspace: the attention slots, then suffix lengths, prefix flags, suffix
+// block table and the prefix partials, each 256-byte aligned.
+struct CascadeWorkspace {
+    size_t slots, sfx_ctx, pflag, sfx_table, pp_o, pp_ml, total;
+};
+CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max_blocks, int num_ctas,
+                                   int splits);
+// p describes the whole call with the caller's block table and lengths; p's
+// workspace pointer is the base of a CascadeWorkspace.
+cudaError_t launch_cascade(const AttnParams &p, const CascadePlan &plan, cudaStream_t stream);
 
 // ------------------------------- kv commit ----------------------------------
 struct CommitLaunch {

@@ -11,7 +11,8 @@ from typing import Optional
 
 import torch
 
-from . import (SvAttnDesc, SvPagedKV, make_accept_desc, make_kv_layers, sv_accept, sv_kv_commit,
+from . import (SvAttnDesc, SvPagedKV, make_accept_desc, make_cascade_desc, make_kv_layers, sv_accept,
+               sv_cascade_attention_workspace_size, sv_cascade_verify_attention, sv_kv_commit,
                sv_verify_attention, sv_verify_attention_workspace_size)
 
 
@@ -41,6 +42,29 @@ class AttentionCall:
 
     def kv_bytes(self) -> int:
         return self.inputs.kv_bytes_unique()
+
+
+class CascadeCall(AttentionCall):
+    """sv_cascade_verify_attention over groups of consecutive sequences whose first
+    prefix_lens[g] keys sit on the group's first member's pages (default: the
+    groups recorded in the inputs)."""
+
+    def __init__(self, a, group_offsets=None, prefix_lens=None, device: str = "cuda",
+                 out: Optional[torch.Tensor] = None, with_status: bool = True):
+        super().__init__(a, device=device, out=out, with_status=with_status)
+        off = a.group_offsets if group_offsets is None else group_offsets
+        pre = a.prefix_lens if prefix_lens is None else prefix_lens
+        if off is None or pre is None:
+            raise ValueError("the inputs carry no groups; pass group_offsets and prefix_lens")
+        self.group_offsets, self.prefix_lens = list(off), list(pre)
+        self.cdesc = make_cascade_desc(self.group_offsets, self.prefix_lens)
+        self.ws_bytes = sv_cascade_attention_workspace_size(self.desc, self.cdesc)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=self.q.device)
+
+    def run(self, stream=None) -> torch.Tensor:
+        sv_cascade_verify_attention(self.desc, self.cdesc, self.q, self.kv, self.block_table, self.ctx_lens,
+                                    self.mask, self.out, self.workspace, self.ws_bytes, self.status, stream)
+        return self.out
 
 
 class AcceptCall:

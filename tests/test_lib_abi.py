@@ -21,6 +21,7 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("sv_verify_attention", "sv_verify_attention_workspace_size", "sv_accept",
+              "sv_cascade_verify_attention", "sv_cascade_attention_workspace_size",
               "sv_status_string", "sv_last_error", "sv_version"):
         assert n in names
 
@@ -85,6 +86,46 @@ def test_attention_rejects_null_and_misaligned_pointers():
 def test_attention_with_no_sequences_is_a_no_op():
     sv.sv_verify_attention(_attn_desc(num_seqs=0), None, sv.SvPagedKV(None, None), None, None, None,
                            None, None, 0)
+
+
+@pytest.mark.parametrize("off,pre", [
+    ([0], []),                       # no groups
+    ([0, 1], [16]),                  # offsets end before num_seqs
+    ([1, 2], [16]),                  # offsets start after 0
+    ([0, 2, 1, 2], [0, 0, 0]),       # decreasing
+    ([0, 1, 2], [16, 8]),            # prefix not whole pages
+    ([0, 1, 2], [-16, 0]),           # negative prefix
+    ([0, 2], [16 * 9]),              # prefix past max_blocks_per_seq pages
+    ([0] * 130 + [2], [0] * 130),    # more than SV_CASCADE_MAX_GROUPS
+])
+def test_cascade_rejects_bad_groups(off, pre):
+    d = _attn_desc()
+    c = sv.make_cascade_desc(off, pre)
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_cascade_verify_attention(d, c, 16, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    assert sv.sv_cascade_attention_workspace_size(d, c) == 0
+
+
+def test_cascade_rejects_bad_descriptors_and_pointers():
+    c = sv.make_cascade_desc([0, 2], [16])
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_cascade_verify_attention(_attn_desc(head_dim=96), c, 16, sv.SvPagedKV(16, 16), 16, 16, None, 16,
+                                       256, 1 << 20)
+    assert e.value.status == sv.SV_ERR_UNSUPPORTED
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_cascade_verify_attention(_attn_desc(), c, 8, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    lib = C.CDLL(sv.library_path())
+    lib.sv_cascade_verify_attention.restype = C.c_int
+    st = lib.sv_cascade_verify_attention(C.byref(_attn_desc()), None, C.c_void_p(16), None, None, None, None,
+                                         None, None, C.c_size_t(0), None, None)
+    assert st == sv.SV_ERR_INVALID_ARG
+
+
+def test_cascade_with_no_sequences_is_a_no_op():
+    sv.sv_cascade_verify_attention(_attn_desc(num_seqs=0), sv.make_cascade_desc([0, 0], [32]), None,
+                                   sv.SvPagedKV(None, None), None, None, None, None, None, 0)
 
 
 @pytest.mark.parametrize("kw,parents,temp,status", [
