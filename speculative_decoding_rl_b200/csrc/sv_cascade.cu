@@ -43,6 +43,7 @@ constexpr int PF_WARPS = CASCADE_ROWS / 16;  // one m16 row block per warp
 constexpr int PF_THREADS = 32 * PF_WARPS;
 constexpr int PREP_THREADS = 128;
 constexpr int MAX_SPLITS = 8;
+constexpr int PF_CTAS_PER_SM = 3;  // resident prefix CTAs per SM (launch bounds; 69.6 KB shared memory each)
 // Running max of a row that has seen no key: finite, so that 2^(M_NONE - m) = 0.
 constexpr float PF_M_NONE = -3.402823466e38f;
 
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(PREP_THREADS) cascade_prep_kernel(const __grid
 }
 
 template <int D>
-__global__ void __launch_bounds__(PF_THREADS, 3) cascade_prefix_kernel(const __grid_constant__ PrefixParams p) {
+__global__ void __launch_bounds__(PF_THREADS, PF_CTAS_PER_SM) cascade_prefix_kernel(const __grid_constant__ PrefixParams p) {
     constexpr int LD = D + 8;                   // padded row: ldmatrix rows land on distinct banks
     constexpr int TILE = CASCADE_KEYS * LD;     // bf16 elements of one K or V tile
     constexpr int NT = CASCADE_KEYS / 8;        // 8-key column blocks of S
@@ -254,12 +255,14 @@ __global__ void __launch_bounds__(PF_THREADS, 3) cascade_prefix_kernel(const __g
             mx[1] = fmaxf(mx[1], fmaxf(sacc[nt][2], sacc[nt][3]));
         }
         float alpha[2];
+        bool raised = false;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
             mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 1));
             mx[k] = fmaxf(mx[k], __shfl_xor_sync(0xffffffffu, mx[k], 2));
             const float mn = fmaxf(mrow[k], mx[k] * sc);
-            alpha[k] = ex2_approx(mrow[k] - mn);  // first tile: 2^(M_NONE - mn) = 0
+            raised |= mn > mrow[k];
+            alpha[k] = ex2_approx(mrow[k] - mn);  // first tile: 2^(M_NONE - mn) = 0; unchanged: 1
             mrow[k] = mn;
         }
         uint32_t pa[NT / 2][4];  // P as A fragments of the PV product
@@ -277,12 +280,14 @@ __global__ void __launch_bounds__(PF_THREADS, 3) cascade_prefix_kernel(const __g
         }
 #pragma unroll
         for (int k = 0; k < 2; ++k) lrow[k] = fmaf(lrow[k], alpha[k], ls[k]);  // this thread's columns only
+        if (__any_sync(0xffffffffu, raised)) {  // an unchanged maximum leaves O as it is (alpha = 1)
 #pragma unroll
-        for (int dn = 0; dn < D / 8; ++dn) {
-            o[dn][0] *= alpha[0];
-            o[dn][1] *= alpha[0];
-            o[dn][2] *= alpha[1];
-            o[dn][3] *= alpha[1];
+            for (int dn = 0; dn < D / 8; ++dn) {
+                o[dn][0] *= alpha[0];
+                o[dn][1] *= alpha[0];
+                o[dn][2] *= alpha[1];
+                o[dn][3] *= alpha[1];
+            }
         }
 
         // O += P V: V tiles [key][dim] read transposed as B fragments
@@ -344,9 +349,11 @@ void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, int num_sms
         base += (rows + CASCADE_ROWS - 1) / CASCADE_ROWS * Hkv;
         max_tiles = max(max_tiles, (pl->pre[g] + CASCADE_KEYS - 1) / CASCADE_KEYS);
     }
-    // Split the prefix only when the (group, head, row chunk) items cannot give
-    // two CTAs per SM: every split adds one partial per row to write and merge.
-    int S = base > 0 ? (2 * num_sms) / base : 1;
+    // The most prefix splits whose items still fit one wave of resident CTAs
+    // (three per SM: shared memory and registers). A second, partial wave costs
+    // more than the latency the extra warps hide: at 448 items for 444 slots the
+    // pass ran longer than at 224. Every split also adds a partial per row.
+    int S = base > 0 ? (PF_CTAS_PER_SM * num_sms) / base : 1;
     S = max(1, min(S, min(MAX_SPLITS, max(1, max_tiles))));
     pl->splits = S;
     int acc = 0;

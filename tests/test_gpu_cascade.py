@@ -65,7 +65,7 @@ def test_members_own_prefix_entries_are_not_read(invalid):
     check(a, off, pre, f"foreign member prefixes (invalid ids: {invalid})")
 
 
-@pytest.mark.parametrize("pre", [[0, 0], [0, 64], [1024, 512]])
+@pytest.mark.parametrize("pre", [[0, 0], [0, 64], [1024, 336]])
 def test_prefix_lengths_and_splits(pre):
     # two small groups on one KV head: few (group, head, chunk) items, so the
     # prefix is split over several CTAs (some splits empty for the short prefix)
