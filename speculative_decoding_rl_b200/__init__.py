@@ -229,10 +229,10 @@ def sv_verify_attention_noalloc(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_
 def make_cascade_desc(group_offsets: Sequence[int], prefix_lens: Sequence[int]) -> SvCascadeDesc:
     """The host-side group description of sv_cascade_verify_attention; it keeps its arrays alive."""
     n = len(prefix_lens)
-    off = (C.c_int32 * (n + 1))(*[int(x) for x in group_offsets])
-    pre = (C.c_int32 * max(n, 1))(*[int(x) for x in prefix_lens])
     if len(group_offsets) != n + 1:
         raise ValueError("group_offsets needs one entry more than prefix_lens")
+    off = (C.c_int32 * (n + 1))(*[int(x) for x in group_offsets])
+    pre = (C.c_int32 * max(n, 1))(*[int(x) for x in prefix_lens])
     d = SvCascadeDesc(n, C.cast(off, C.POINTER(C.c_int32)), C.cast(pre, C.POINTER(C.c_int32)))
     d._keep = (off, pre)
     return d

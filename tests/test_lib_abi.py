@@ -123,6 +123,16 @@ def test_cascade_rejects_bad_descriptors_and_pointers():
     assert st == sv.SV_ERR_INVALID_ARG
 
 
+def test_cascade_desc_needs_one_offset_per_group_boundary():
+    with pytest.raises(ValueError):
+        sv.make_cascade_desc([0, 1], [16, 16])
+    with pytest.raises(ValueError):
+        sv.make_cascade_desc([0, 1, 2, 3], [16, 16])
+    d = sv.make_cascade_desc([0, 3, 5], [32, 0])
+    assert d.num_groups == 2 and [d.group_offsets[i] for i in range(3)] == [0, 3, 5]
+    assert [d.prefix_lens[i] for i in range(2)] == [32, 0]
+
+
 def test_cascade_with_no_sequences_is_a_no_op():
     sv.sv_cascade_verify_attention(_attn_desc(num_seqs=0), sv.make_cascade_desc([0, 0], [32]), None,
                                    sv.SvPagedKV(None, None), None, None, None, None, None, 0)
