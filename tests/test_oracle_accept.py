@@ -12,7 +12,9 @@ What fixes the rule without an implementation to compare against:
     a one-hot q at d accepts with probability p(d) and then resamples p with d
     removed; T = 0 accepts exactly up to the first mismatch with argmax; a tree
     in which every node has at most one child equals the chain;
-  * the inverse CDF equals numpy's searchsorted on the cumulative sum.
+  * the inverse CDF equals numpy's searchsorted on the cumulative sum;
+  * work on top of a rejected draft is discarded (TLT reading notes, "1. RL and
+    SD"): nothing after the first rejection changes the result.
 """
 import numpy as np
 import pytest
@@ -172,6 +174,31 @@ def test_greedy_accepts_up_to_first_argmax_mismatch():
         k = r.accept_len[b]
         assert r.accept_path[b, :k].tolist() == list(range(1, k + 1))
         assert (r.accept_path[b, k:] == -1).all()
+
+
+@pytest.mark.parametrize("T", [1.0, 0.7, 0.0])
+def test_outputs_ignore_everything_after_the_first_rejection(T):
+    """Work on top of a rejected draft is discarded (TLT reading notes, "1. RL and SD"):
+    replacing every later draft token, draft row and target row changes nothing."""
+    N, V = 7, 200
+    a = W.make_accept_inputs(256, N, V, seed=41, logit_std=2.0, draft_noise=1.5, temperature=T)
+    l, q, d = a.target_logits.numpy(), a.draft_probs.numpy(), a.draft_tokens.numpy()
+    r = oracle.accept(l, q, d, T, seed=5)
+    rng = np.random.default_rng(6)
+    l2, q2, d2 = l.copy(), q.copy(), d.copy()
+    rejected = 0
+    for b in range(l.shape[0]):
+        k = int(r.accept_len[b])  # drafts 1..k accepted, draft k+1 (column k) rejected
+        if k == N - 1:
+            continue
+        rejected += 1
+        l2[b, k + 1:] = rng.normal(0, 3, size=l2[b, k + 1:].shape)       # target rows after node k
+        q2[b, k + 1:] = rng.dirichlet(np.ones(V), size=N - 2 - k)         # drafts k+2 .. N-1
+        d2[b, k + 1:] = rng.integers(0, V, size=N - 2 - k)
+    r2 = oracle.accept(l2, q2, d2, T, seed=5)
+    assert rejected > 50
+    for name in ("accept_len", "accept_path", "next_token", "tie_depth", "tie_draw", "flags"):
+        np.testing.assert_array_equal(getattr(r, name), getattr(r2, name))
 
 
 def test_greedy_lowest_index_on_ties():
