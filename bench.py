@@ -387,6 +387,11 @@ def run_ours(args, world, rank, local):
     accepted = float((lens_out[Wm:Wm + K].to(torch.int64) + 1).sum().item())
     accepted_total = sum_over_ranks(accepted, world)
     tok_s = accepted_total / elapsed_max
+    # the timed steps' accept statistics (this rank): a step is "effective" when it
+    # accepted at least one draft
+    timed_lens = lens_out[Wm:Wm + K].to(torch.float64)
+    accept_stats = {"draft_len": N - 1, "mean_accept_len": float(timed_lens.mean().item()),
+                    "effective_percent": 100.0 * float((timed_lens >= 1).to(torch.float64).mean().item())}
 
     # accept-call timing
     ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -506,7 +511,7 @@ def run_ours(args, world, rank, local):
                        "l2": ("inputs larger than L2 (every layer has its own KV pool)" if n_pools == layers else
                               f"inputs larger than L2 ({n_pools} KV pools of {pool_bytes / 1e9:.1f} GB cycled over {layers} layers)"),
                        "parallelism": f"replicas x{world}"},
-            "accepted_tok_s": tok_s,
+            "accepted_tok_s": tok_s, "accept_stats": accept_stats,
             "t_attn_call_ms": 1e3 * t_attn, "t_accept_call_ms": 1e3 * t_acc,
             "t_attn_plain_call_ms": None if t_plain is None else 1e3 * t_plain,
             "hbm_gbs_step": step_bytes / (elapsed_max / K) / 1e9,
