@@ -244,6 +244,11 @@ SV_API sv_status sv_accept(const sv_accept_desc *desc, const float *target_logit
  * accept_len or path is malformed (SV_FLAG_BAD_PATH). Every source row is read
  * before any row is written, so overlapping moves are safe. Limits: D a
  * multiple of 8 up to 256, N <= 64. Pools 16-byte aligned.
+ * new_ctx_lens and status_flags are written while the other CTAs of a
+ * sequence still read the inputs, so neither may overlap block_table,
+ * ctx_lens, accept_len, accept_path or each other (an in-place update of
+ * ctx_lens is refused with SV_ERR_INVALID_ARG before any launch; use a
+ * second buffer).
  * The pages have no interface for this step; its arguments follow the verify
  * and accept calls whose results it applies.
  */
@@ -419,7 +424,8 @@ SV_API double sv_ctl_acceptance(const sv_ctl *ctl);
  * (sv_verify_attention_workspace_size) exceeds the scratch is refused with
  * SV_ERR_WORKSPACE before any launch.
  * The first call on a device looks up that device's scratch address; make it
- * before any stream capture. All calls on a device share the scratch, which
+ * before any stream capture (a lookup that fails returns SV_ERR_CUDA and is
+ * retried by the next call). All calls on a device share the scratch, which
  * keeps the last call's contents (nothing in it needs clearing); calls whose
  * executions overlap on the GPU race on it and must be ordered by the caller.
  */

@@ -43,6 +43,8 @@ def lib() -> C.CDLL:
         i32, u32, u64, f64 = C.c_int, C.c_uint32, C.c_uint64, C.c_double
         L.orc_philox4x32_10.argtypes = [P, P, P]
         L.orc_philox4x32_10.restype = None
+        L.orc_philox4x32_10_many.argtypes = [C.c_long, P, P, P]
+        L.orc_philox4x32_10_many.restype = None
         L.orc_uniform.argtypes = [u64, u32, u32, u32, u32]
         L.orc_uniform.restype = f64
         L.orc_attention.argtypes = [i32] * 8 + [P] * 8
@@ -83,6 +85,15 @@ def philox4x32_10(ctr: Sequence[int], key: Sequence[int]) -> np.ndarray:
     k = np.asarray(key, dtype=np.uint32)
     out = np.zeros(4, dtype=np.uint32)
     lib().orc_philox4x32_10(_p(c), _p(k), _p(out))
+    return out
+
+
+def philox4x32_10_many(ctrs: np.ndarray, key: Sequence[int]) -> np.ndarray:
+    """The block function of every row of ``ctrs`` (uint32 [n][4]) under ``key`` (two words)."""
+    c = np.ascontiguousarray(ctrs, dtype=np.uint32).reshape(-1, 4)
+    k = np.asarray(key, dtype=np.uint32)
+    out = np.zeros_like(c)
+    lib().orc_philox4x32_10_many(len(c), _p(c), _p(k), _p(out))
     return out
 
 

@@ -73,6 +73,12 @@ void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
     out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
+/* The block function applied to n counters (ctr and out: [n][4]) under one key. */
+void orc_philox4x32_10_many(long n, const uint32_t *ctr, const uint32_t key[2], uint32_t *out)
+{
+    for (long i = 0; i < n; ++i) orc_philox4x32_10(ctr + 4 * i, key, out + 4 * i);
+}
+
 double orc_uniform(uint64_t seed, uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3)
 {
     uint32_t ctr[4] = {c0, c1, c2, c3};

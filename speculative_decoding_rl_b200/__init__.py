@@ -20,6 +20,7 @@ __all__ = [
     "SvCascadeDesc", "make_cascade_desc", "sv_cascade_attention_workspace_size", "sv_cascade_verify_attention",
     "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig", "SvHistoryDesc", "sv_history_draft",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
+    "sv_testing_philox4x32_10", "sv_testing_verify_attention_stalled", "SV_FLAG_TIMEOUT",
     "SV_FLAG_NONFINITE", "SV_FLAG_BAD_CONTEXT", "SV_FLAG_BAD_TOKEN", "SV_FLAG_BAD_BLOCK",
 ]
 
@@ -139,6 +140,11 @@ def _load() -> C.CDLL:
     L.sv_ctl_acceptance.restype = C.c_double
     L.sv_history_draft.argtypes = [C.POINTER(SvHistoryDesc)] + [P] * 10 + [P]
     L.sv_history_draft.restype = C.c_int
+    L.sv_testing_philox4x32_10.argtypes = [u64, P, P, C.c_int64, P]
+    L.sv_testing_philox4x32_10.restype = C.c_int
+    L.sv_testing_verify_attention_stalled.argtypes = [C.POINTER(SvAttnDesc), P, C.POINTER(SvPagedKV), P, P, P, P,
+                                                      P, sz, P, u64, P]
+    L.sv_testing_verify_attention_stalled.restype = C.c_int
     L.sv_status_string.argtypes = [C.c_int]
     L.sv_status_string.restype = C.c_char_p
     L.sv_last_error.argtypes = []
@@ -281,6 +287,23 @@ def sv_history_draft(desc: SvHistoryDesc, history_tokens, history_lens, history_
     _check(_L().sv_history_draft(C.byref(desc), _ptr(history_tokens), _ptr(history_lens), _ptr(history_reward),
                                  _ptr(history_group), _ptr(seq_tokens), _ptr(seq_lens), _ptr(seq_group),
                                  _ptr(draft_tokens), _ptr(draft_len), _ptr(draft_probs), _stream(stream)))
+
+
+def sv_testing_philox4x32_10(key: int, counters, out, n: int, stream=None) -> None:
+    """Test hook: the device Philox4x32-10 words of n counters (uint32 [n][4] each)."""
+    _check(_L().sv_testing_philox4x32_10(int(key) & 0xFFFFFFFFFFFFFFFF, _ptr(counters), _ptr(out), int(n),
+                                         _stream(stream)))
+
+
+def sv_testing_verify_attention_stalled(desc: SvAttnDesc, q, paged_kv: SvPagedKV, block_table, ctx_lens,
+                                        draft_mask, out, workspace, workspace_bytes: int, status_flags,
+                                        wait_limit_ns: int, stream=None) -> None:
+    """Test hook: sv_verify_attention with one wait per CTA made to run out after
+    wait_limit_ns; every sequence comes back flagged SV_FLAG_TIMEOUT."""
+    _check(_L().sv_testing_verify_attention_stalled(C.byref(desc), _ptr(q), C.byref(paged_kv), _ptr(block_table),
+                                                    _ptr(ctx_lens), _ptr(draft_mask), _ptr(out), _ptr(workspace),
+                                                    int(workspace_bytes), _ptr(status_flags), int(wait_limit_ns),
+                                                    _stream(stream)))
 
 
 def default_ctl_config() -> SvCtlConfig:

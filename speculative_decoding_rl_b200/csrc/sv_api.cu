@@ -21,6 +21,13 @@ sv_status fail(sv_status s, const char *fmt, ...) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// True when the byte ranges [a, a+na) and [b, b+nb) share a byte.
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    if (!a || !b || na == 0 || nb == 0) return false;
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
 sv_status check_attn_desc(const sv_attn_desc *d) {
     if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
     if (d->num_seqs < 0) return fail(SV_ERR_INVALID_ARG, "num_seqs < 0");
@@ -100,6 +107,8 @@ sv::AttnParams attn_params(const sv_attn_desc *d, const void *q, const sv_paged_
     p.num_ctas = ctas;
     p.scale_log2 = (float)(1.4426950408889634 / sqrt((double)p.D));
     p.ws_partial = static_cast<float *>(workspace);
+    p.wait_limit_ns = 2000000000ull;
+    p.stall = 0;
     return p;
 }
 
@@ -138,6 +147,19 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
                               const int32_t *block_table, const int32_t *ctx_lens,
                               const uint64_t *draft_mask, void *out, void *workspace,
                               size_t workspace_bytes, int32_t *status_flags, void *stream) {
+    return sv::verify_attention_entry(d, q, kv, block_table, ctx_lens, draft_mask, out, workspace,
+                                      workspace_bytes, status_flags, stream, 2000000000ull, 0);
+}
+
+}  // extern "C"
+
+namespace sv {
+
+sv_status verify_attention_entry(const sv_attn_desc *d, const void *q, const sv_paged_kv *kv,
+                                 const int32_t *block_table, const int32_t *ctx_lens,
+                                 const uint64_t *draft_mask, void *out, void *workspace,
+                                 size_t workspace_bytes, int32_t *status_flags, void *stream,
+                                 uint64_t wait_limit_ns, int stall) {
     sv_status s = check_attn_desc(d);
     if (s != SV_OK) return s;
     if (d->num_seqs == 0) return SV_OK;
@@ -149,12 +171,18 @@ sv_status sv_verify_attention(const sv_attn_desc *d, const void *q, const sv_pag
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
         return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);
 
-    const sv::AttnParams p =
+    sv::AttnParams p =
         attn_params(d, q, kv, block_table, ctx_lens, draft_mask, out, workspace, status_flags, ctas);
+    p.wait_limit_ns = wait_limit_ns;
+    p.stall = stall;
     cudaError_t e = sv::launch_attention(p, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(SV_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
     return SV_OK;
 }
+
+}  // namespace sv
+
+extern "C" {
 
 size_t sv_cascade_attention_workspace_size(const sv_attn_desc *d, const sv_cascade_desc *c) {
     if (check_attn_desc(d) != SV_OK || check_cascade_desc(d, c) != SV_OK) return 0;
@@ -266,6 +294,21 @@ sv_status sv_kv_commit(const sv_attn_desc *d, int32_t num_layers, const sv_kv_la
     if (!aligned(block_table, 4) || !aligned(ctx_lens, 4) || !aligned(accept_len, 4) || !aligned(new_ctx_lens, 4) ||
         (accept_path && !aligned(accept_path, 4)) || (status_flags && !aligned(status_flags, 4)))
         return fail(SV_ERR_INVALID_ARG, "misaligned pointer");
+    {
+        // every CTA of a sequence reads its table row, length, accept length and
+        // path while one of them writes the new length and the status: the
+        // outputs must not alias any input (an in-place length update would let
+        // late CTAs read the new length)
+        const size_t B4 = (size_t)d->num_seqs * 4;
+        const void *in[] = {block_table, ctx_lens, accept_len, accept_path};
+        const size_t in_bytes[] = {B4 * (size_t)d->max_blocks_per_seq, B4, B4,
+                                   B4 * (size_t)(d->num_q_rows > 1 ? d->num_q_rows - 1 : 1)};
+        for (int i = 0; i < 4; ++i)
+            if (overlaps(new_ctx_lens, B4, in[i], in_bytes[i]) || overlaps(status_flags, B4, in[i], in_bytes[i]))
+                return fail(SV_ERR_INVALID_ARG, "new_ctx_lens and status_flags must not overlap an input array");
+        if (overlaps(new_ctx_lens, B4, status_flags, B4))
+            return fail(SV_ERR_INVALID_ARG, "new_ctx_lens and status_flags overlap");
+    }
     sv::CommitLaunch c;
     memset(&c, 0, sizeof c);
     c.block_table = block_table;

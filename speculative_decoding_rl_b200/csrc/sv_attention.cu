@@ -63,7 +63,10 @@ __host__ __device__ constexpr int tc_threads(int RP) { return 32 * (WARPS_PER_WG
 // that s*scale - M_NONE is +huge for a visible score (it votes for a raise) and
 // -inf for a masked one (p = 0), with no special case in the exponentials.
 constexpr float M_NONE = -3.402823466e38f;
-constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait, then the kernel gives up
+// Drain limit: after an abort, a role still waits this long for its own copies
+// and products in flight. The limit of every other wait is AttnParams::wait_limit_ns
+// (2 s; test hooks shorten it).
+constexpr uint64_t WAIT_LIMIT_NS = 2000000000ull;
 
 // ---------------------------------------------------------------------------
 // Schedule helpers (attention and combine kernels agree on these).
@@ -197,7 +200,6 @@ struct TcParams {
     CUtensorMap tm_q;
     AttnParams a;
     int NK, NV, NP, NQ, Nc;  // K / V / P slots, query buffers (1 or 2), query rows per chunk
-    uint32_t epoch;
 };
 
 // ---------------------------------------------------------------------------
@@ -246,6 +248,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     float *mfin = reinterpret_cast<float *>(base + L.off_mfin); // [RP] its row maxima
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
+    uint64_t *stall_bar = reinterpret_cast<uint64_t *>(base + L.off_misc + 8);  // test hook: never arrived on
     int *scratch = reinterpret_cast<int *>(base + L.off_misc + 16);  // one int per warp (<= 28), used once
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         mbar_init(done_bar, 1);
         for (int s = 0; s < NV; ++s) mbar_init(&vz[s], 1);
         for (int g = 0; g < NWG; ++g) mbar_init(&wg_bar[g], WARPS_PER_WG);
+        mbar_init(stall_bar, 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -323,7 +327,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 if (is_k && (lt == 0 || ti.j == 0)) {
                     ++lu;
                     const int qb = qbuf(lu);
-                    if (!mbar_wait(&q_empty[qb], qphase(lu) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                    if (!mbar_wait(&q_empty[qb], qphase(lu) ^ 1, abort_flag, p.wait_limit_ns)) break;
                     mbar_arrive_expect_tx(&q_full[qb], q_box_bytes * nDA);
                     uint8_t *qdst = base + L.off_q + qb * L.q_bytes;
                     for (int a = 0; a < nDA; ++a)
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                                     ti.b * p.N + rc * P.Nc);
                 }
                 const int s = lt % NR;
-                if (!mbar_wait(&empty[s], ((lt / NR) & 1) ^ 1, abort_flag, WAIT_LIMIT_NS)) break;
+                if (!mbar_wait(&empty[s], ((lt / NR) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&full[s], L.tile_bytes);
                 uint8_t *dst = ring + s * L.tile_bytes;
 #pragma unroll
@@ -385,7 +389,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
             const int s = lt % NV;
             const uint32_t par = (lt / NV) & 1;
-            const bool landed = mbar_test(&v_full[s], par) || mbar_wait(&v_full[s], par, abort_flag, WAIT_LIMIT_NS);
+            const bool landed = mbar_test(&v_full[s], par) || mbar_wait(&v_full[s], par, abort_flag, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, landed)) break;
             const int k0 = max(0, CL[ti.b] - ti.j * TILE_KEYS);  // first key of the tile past ctx_len
             if (k0 < TILE_KEYS) {
@@ -474,7 +478,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     if (*abort_flag) break;
                     const uint64_t now = globaltimer_ns();
                     if (idle == 64) idle_since = now;
-                    else if (now - idle_since > WAIT_LIMIT_NS) { *abort_flag = 1; break; }
+                    else if (now - idle_since > p.wait_limit_ns) { *abort_flag = 1; break; }
                 }
             }
             mma_commit(done_bar);  // every MMA of this CTA has finished before TMEM is freed
@@ -504,7 +508,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         };
         // warp-uniform bounded wait: the tcgen05 accesses that follow are .sync.aligned
         auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
-            const bool r = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, WAIT_LIMIT_NS);
+            const bool r = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, p.wait_limit_ns);
             return __all_sync(0xffffffffu, r);
         };
         auto wg_sync = [&]() -> bool {
@@ -591,6 +595,11 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             }
             return true;
         };
+
+        // Test hook (p.stall): wait on a barrier nothing arrives on, so that the
+        // bounded wait runs out, the CTA aborts through the same path as a real
+        // timeout and every sequence is flagged SV_FLAG_TIMEOUT.
+        if (p.stall) ok = wait_w(stall_bar, 0);
 
         // one pass past the last tile closes and finishes the CTA's last unit
         TileInfo tnext = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
@@ -1044,11 +1053,6 @@ static cudaError_t launch_tc_rp(TcParams &P, int RP, cudaStream_t stream) {
     return cudaErrorInvalidValue;
 }
 
-static uint32_t next_epoch() {
-    static std::atomic<uint32_t> e{0x5A000000u};
-    return ++e;
-}
-
 cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     TcParams P;
     memset(&P, 0, sizeof P);
@@ -1056,7 +1060,6 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     int RU, RC, Nc;
     row_chunks(p.N, p.G, &RU, &RC, &Nc);
     P.Nc = Nc;
-    P.epoch = next_epoch();
     if (!encode_pool_map(&P.tm_k, p.k_pool, p.num_blocks, p.Hkv, p.D) ||
         !encode_pool_map(&P.tm_v, p.v_pool, p.num_blocks, p.Hkv, p.D) ||
         !encode_q_map(&P.tm_q, p.q, p.B, p.N, p.Hq, p.D, p.G, Nc))

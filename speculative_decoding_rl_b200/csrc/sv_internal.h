@@ -61,6 +61,10 @@ struct AttnParams {
     const float *pp_ml;        // [pp_splits][B][N][Hq][2] running max (log2 domain), row sum
     const int32_t *pflag;      // [B] status bits found on the prefix pages
     int pp_splits;
+    // Bound of every device-side wait (2 s). Test hooks shorten it, and with
+    // stall set make one wait per CTA run out (see sv_testing_*).
+    uint64_t wait_limit_ns;
+    int stall;
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
@@ -117,5 +121,12 @@ cudaError_t launch_history_draft(const HistoryLaunch &h, cudaStream_t stream);
 
 // Sets the text sv_last_error() returns on the calling thread.
 void record_error(const char *msg);
+
+// sv_verify_attention with its wait bound and the stall test hook exposed.
+sv_status verify_attention_entry(const sv_attn_desc *d, const void *q, const sv_paged_kv *kv,
+                                 const int32_t *block_table, const int32_t *ctx_lens,
+                                 const uint64_t *draft_mask, void *out, void *workspace,
+                                 size_t workspace_bytes, int32_t *status_flags, void *stream,
+                                 uint64_t wait_limit_ns, int stall);
 
 }  // namespace sv

@@ -13,7 +13,9 @@
 //
 // Set-up: the first call on each device looks up that device's copy of the
 // scratch array (cudaGetSymbolAddress, with the device current) and caches
-// the address; make that first call before any stream capture. All calls on
+// the address; make that first call before any stream capture. A lookup that
+// fails is not cached: the call returns SV_ERR_CUDA and the next call tries
+// again. All calls on
 // a device share the one array and it keeps whatever the last call left in
 // it; the kernels write every scratch word before they read it, so nothing
 // needs clearing. Two calls whose executions overlap on the GPU (on different
@@ -31,9 +33,25 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SV_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_once[kMaxDevices];
-void *g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_lookup_mutex;
+void *g_scratch_ptr[kMaxDevices];  // set once a lookup on that device succeeded
+
+// The address of `dev`'s copy of the scratch array (dev is current), or null.
+// Only a successful lookup is kept: a failed one (say, made while a stream was
+// being captured) is retried by the next call, and its error is cleared from
+// the runtime so that it is not reported later as another call's failure.
+void *scratch_address(int dev) {
+    std::lock_guard<std::mutex> lock(g_lookup_mutex);
+    if (g_scratch_ptr[dev] == nullptr) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) == cudaSuccess) {
+            g_scratch_ptr[dev] = ptr;
+        } else {
+            (void)cudaGetLastError();
+        }
+    }
+    return g_scratch_ptr[dev];
+}
 
 }  // namespace
 
@@ -46,11 +64,9 @@ extern "C" sv_status sv_verify_attention_noalloc(const sv_attn_desc *desc, const
         sv::record_error("cannot query the current device");
         return SV_ERR_CUDA;
     }
-    std::call_once(g_once[dev], [dev] {
-        // the caller's current device is `dev`; the symbol's address is per device
-        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_noalloc_scratch);
-    });
-    if (g_scratch_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) {
+    // the caller's current device is `dev`; the symbol's address is per device
+    void *scratch = scratch_address(dev);
+    if (scratch == nullptr) {
         sv::record_error("cannot look up the scratch array on the current device");
         return SV_ERR_CUDA;
     }
@@ -64,5 +80,5 @@ extern "C" sv_status sv_verify_attention_noalloc(const sv_attn_desc *desc, const
         return SV_ERR_WORKSPACE;
     }
     return sv_verify_attention(desc, q, paged_kv, block_table, ctx_lens, draft_mask, out,
-                               g_scratch_ptr[dev], SV_NOALLOC_SCRATCH_BYTES, status_flags, stream);
+                               scratch, SV_NOALLOC_SCRATCH_BYTES, status_flags, stream);
 }

@@ -10,17 +10,20 @@ import pytest
 import speculative_decoding_rl_b200 as sv
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "specverify.h")
+HEADERS = [os.path.join(ROOT, "include", h) for h in ("specverify.h", "specverify_testing.h")]
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    return sorted(set(re.findall(r"SV_API\s+[\w\s\*]*?\b(sv_\w+)\s*\(", text)))
+    names = set()
+    for h in HEADERS:
+        names.update(re.findall(r"SV_API\s+[\w\s\*]*?\b(sv_\w+)\s*\(", open(h).read()))
+    return sorted(names)
 
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("sv_verify_attention", "sv_verify_attention_workspace_size", "sv_accept",
+              "sv_testing_philox4x32_10", "sv_testing_verify_attention_stalled",
               "sv_cascade_verify_attention", "sv_cascade_attention_workspace_size",
               "sv_status_string", "sv_last_error", "sv_version"):
         assert n in names
@@ -35,11 +38,12 @@ def test_library_exports_every_declared_symbol():
         assert n in exported, n
 
 
-def test_library_targets_sm100a_only():
-    out = subprocess.check_output(["/usr/local/cuda/bin/cuobjdump", "--list-elf", sv.library_path()],
-                                  text=True)
-    archs = set(re.findall(r"sm_\w+", out))
-    assert archs == {"sm_100a"}, archs
+def test_library_is_built_for_sm100a_only():
+    from speculative_decoding_rl_b200 import build
+    flags = build.NVCC_FLAGS
+    targets = [flags[i + 1] for i, f in enumerate(flags) if f == "-gencode"]
+    assert targets == ["arch=compute_100a,code=sm_100a"], targets
+    assert not any(f.startswith("-arch") or f.startswith("--gpu-architecture") for f in flags)
 
 
 def test_status_strings_and_version():
@@ -216,3 +220,46 @@ def test_history_draft_rejects_null_and_misaligned_pointers():
     with pytest.raises(sv.SvError):
         sv.sv_history_draft(d, 64, 64, 66, 64, 64, 64, 64, 64, 64, 64)
     sv.sv_history_draft(sv.SvHistoryDesc(0, 3, 16, 16, 3, 4, 0), 0, 0, 0, 0, 0, 0, 0, 0, 0)
+
+
+def test_kv_commit_refuses_outputs_that_alias_inputs():
+    # an in-place length update (new_ctx_lens == ctx_lens) would let late CTAs
+    # read the new length; it is refused on the host before any launch
+    d = sv.SvAttnDesc(4, 5, 4, 2, 128, 16, 4, 8)
+    base = dict(block_table=0x10000, ctx_lens=0x20000, accept_len=0x30000, accept_path=0x40000,
+                new_ctx_lens=0x50000, status_flags=0x60000)
+    for out_name in ("new_ctx_lens", "status_flags"):
+        for in_name in ("block_table", "ctx_lens", "accept_len", "accept_path"):
+            for delta in (0, 4, 12):
+                args = dict(base)
+                args[out_name] = base[in_name] + delta
+                with pytest.raises(sv.SvError) as e:
+                    sv.sv_kv_commit(d, [(256, 512)], args["block_table"], args["ctx_lens"], args["accept_len"],
+                                    args["accept_path"], args["new_ctx_lens"], args["status_flags"])
+                assert e.value.status == sv.SV_ERR_INVALID_ARG, (out_name, in_name, delta)
+                assert "overlap" in sv.sv_last_error()
+    args = dict(base)
+    args["status_flags"] = base["new_ctx_lens"] + 8
+    with pytest.raises(sv.SvError):
+        sv.sv_kv_commit(d, [(256, 512)], *[args[k] for k in ("block_table", "ctx_lens", "accept_len", "accept_path",
+                                                             "new_ctx_lens", "status_flags")])
+
+
+def test_testing_hooks_reject_bad_arguments():
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_testing_philox4x32_10(0, 16, 16, -1, stream=0)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError) as e:
+        sv.sv_testing_philox4x32_10(0, 8, 16, 4, stream=0)
+    assert e.value.status == sv.SV_ERR_INVALID_ARG
+    sv.sv_testing_philox4x32_10(0, None, None, 0, stream=0)  # nothing to do
+    d = _attn_desc()
+    for lim in (0, 2_000_000_001):
+        with pytest.raises(sv.SvError) as e:
+            sv.sv_testing_verify_attention_stalled(d, 16, sv.SvPagedKV(16, 16), 16, 16, None, 16, 256, 1 << 20,
+                                                   None, lim, stream=0)
+        assert e.value.status == sv.SV_ERR_INVALID_ARG
+    with pytest.raises(sv.SvError) as e:  # descriptor checks as for the plain call
+        sv.sv_testing_verify_attention_stalled(_attn_desc(head_dim=96), 16, sv.SvPagedKV(16, 16), 16, 16, None, 16,
+                                               256, 1 << 20, None, 10_000_000, stream=0)
+    assert e.value.status == sv.SV_ERR_UNSUPPORTED

@@ -54,3 +54,16 @@ def test_counter_words_and_key_all_matter():
     assert oracle.uniform(5, 1, 2, 1, 0) != base
     assert oracle.uniform(6, 1, 2, 0, 0) != base
     assert oracle.uniform(5 + (1 << 32), 1, 2, 0, 0) != base
+
+
+def test_many_counters_equals_one_at_a_time():
+    rng = np.random.default_rng(11)
+    ctrs = rng.integers(0, 2**32, size=(64, 4), dtype=np.uint64).astype(np.uint32)
+    key = [0x9E3779B9, 0xDEADBEEF]
+    many = oracle.philox4x32_10_many(ctrs, key)
+    for i in range(len(ctrs)):
+        assert list(many[i]) == list(oracle.philox4x32_10(ctrs[i], key))
+    # and the known answers through the batched entry
+    rows = _kat()
+    for ctr, key, want in rows:
+        assert [int(x) for x in oracle.philox4x32_10_many(np.array([ctr]), key)[0]] == want

@@ -3,16 +3,16 @@ cannot allocate device memory (it uses the library's built-in scratch array
 instead of a workspace argument).
 
 Checks, through the C-ABI, that two calls in a row give the same results as
-sv_verify_attention with a caller-provided workspace, within the attention
-tolerance the other tests use, and that a request larger than the built-in
-scratch is refused before anything runs. Collected last on purpose.
+sv_verify_attention with a caller-provided workspace, bit for bit (the same
+kernels on the same inputs are deterministic; only where the partials live
+differs), and that a request larger than the built-in scratch is refused
+before anything runs. Collected last on purpose.
 """
 import numpy as np
 import pytest
 import torch
 
 import speculative_decoding_rl_b200 as sv
-from parity import assert_attention_close
 from speculative_decoding_rl_b200 import workloads as W
 from speculative_decoding_rl_b200.session import AttentionCall
 
@@ -25,7 +25,7 @@ def _noalloc(call: AttentionCall):
     sv.sv_verify_attention_noalloc(call.desc, call.q, call.kv, call.block_table, call.ctx_lens, call.mask,
                                    out, status)
     torch.cuda.synchronize()
-    return out.float().cpu().numpy(), status.cpu().numpy()
+    return out.view(torch.int16).cpu().numpy(), status.cpu().numpy()
 
 
 def test_noalloc_matches_workspace_entry_point_twice():
@@ -36,14 +36,14 @@ def test_noalloc_matches_workspace_entry_point_twice():
     ]
     for a in cases:
         call = AttentionCall(a)
-        ref = call.run().float().cpu().numpy()
+        ref = call.run().view(torch.int16).cpu().numpy()
         torch.cuda.synchronize()
         ref_status = call.status.cpu().numpy()
         assert sv.sv_verify_attention_workspace_size(call.desc) <= sv.SV_NOALLOC_SCRATCH_BYTES
         for _ in range(2):  # the scratch keeps the previous call's contents
             got, status = _noalloc(call)
             np.testing.assert_array_equal(status, ref_status)
-            assert_attention_close(got, ref, "noalloc vs workspace entry point")
+            np.testing.assert_array_equal(got, ref)  # bf16 bits of every output
 
 
 def test_noalloc_refuses_requests_beyond_the_scratch():
