@@ -181,6 +181,9 @@ SV_API sv_status sv_cascade_verify_attention(const sv_attn_desc *desc, const sv_
  *   next_token    int32 [B]        out: the token emitted after the accepted path
  *   accept_path   int32 [B][N-1] or NULL   out: accepted node ids, then -1
  *   status_flags  int32 [B] or NULL        out: SV_FLAG_* bits
+ *   workspace     device memory of sv_accept_workspace_size(desc) bytes, 256-byte
+ *                 aligned; nothing in it needs clearing (every word is written
+ *                 before it is read); calls sharing it must not overlap
  * tree_parents is a HOST array of N entries (tree_parents[0] = -1,
  * 0 <= tree_parents[c] < c), copied at the call; NULL = chain (parent c-1).
  *
@@ -201,7 +204,13 @@ SV_API sv_status sv_cascade_verify_attention(const sv_attn_desc *desc, const sv_
  * sum_{y<=x} w(y) > u * sum(w), else the last x with w(x) > 0.
  * Arithmetic is fp32. A sequence flagged SV_FLAG_NONFINITE gets
  * accept_len 0, next_token 0; a bad draft token counts as rejected.
- * Limits: 1 <= N <= 64, 1 <= V <= 450560 (8 x 56320), 0 <= B <= 65535.
+ * The work is spread over every SM: one pass reads every logit once for the
+ * row statistics, a per-sequence walk takes the decisions, and each rejection
+ * (a chain has one, a tree at most its worst walk's count) costs one more pass
+ * over that node's logit row and the rejected children's draft rows; the draw
+ * re-reads one slice of 8192 entries. The kernels follow one another on
+ * `stream` with no device-side wait of their own.
+ * Limits: 1 <= N <= 64, 1 <= V <= 4194304, 0 <= B <= 65535.
  */
 typedef struct {
     int32_t num_seqs;             /* B */
@@ -210,10 +219,13 @@ typedef struct {
     const int32_t *tree_parents;  /* HOST [N] or NULL (chain) */
 } sv_accept_desc;
 
+/* Bytes of device workspace sv_accept needs for `desc`; 0 on an invalid desc. */
+SV_API size_t sv_accept_workspace_size(const sv_accept_desc *desc);
+
 SV_API sv_status sv_accept(const sv_accept_desc *desc, const float *target_logits, const float *draft_probs,
                     const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
                     int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
-                    int32_t *status_flags, void *stream);
+                    int32_t *status_flags, void *workspace, size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------
  * KV commit after accept

@@ -17,6 +17,7 @@ from typing import Optional, Sequence
 __all__ = [
     "SvError", "SvAttnDesc", "SvPagedKV", "SvAcceptDesc", "SvKVLayer",
     "sv_verify_attention_workspace_size", "sv_verify_attention", "sv_verify_attention_noalloc", "sv_accept",
+    "sv_accept_workspace_size",
     "SvCascadeDesc", "make_cascade_desc", "sv_cascade_attention_workspace_size", "sv_cascade_verify_attention",
     "sv_kv_commit", "make_kv_layers", "SdController", "SvCtlConfig", "SvHistoryDesc", "sv_history_draft",
     "sv_status_string", "sv_last_error", "sv_version", "library_path",
@@ -122,7 +123,9 @@ def _load() -> C.CDLL:
     L.sv_cascade_verify_attention.argtypes = [C.POINTER(SvAttnDesc), C.POINTER(SvCascadeDesc), P,
                                               C.POINTER(SvPagedKV), P, P, P, P, P, sz, P, P]
     L.sv_cascade_verify_attention.restype = C.c_int
-    L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P]
+    L.sv_accept_workspace_size.argtypes = [C.POINTER(SvAcceptDesc)]
+    L.sv_accept_workspace_size.restype = sz
+    L.sv_accept.argtypes = [C.POINTER(SvAcceptDesc), P, P, P, f32, u64, P, P, P, P, P, sz, P]
     L.sv_accept.restype = C.c_int
     L.sv_kv_commit.argtypes = [C.POINTER(SvAttnDesc), i32, C.POINTER(SvKVLayer), P, P, P, P, P, P, P]
     L.sv_kv_commit.restype = C.c_int
@@ -259,12 +262,17 @@ def sv_cascade_verify_attention(desc: SvAttnDesc, cdesc: SvCascadeDesc, q, paged
                                             _stream(stream)))
 
 
+def sv_accept_workspace_size(desc: SvAcceptDesc) -> int:
+    return int(_L().sv_accept_workspace_size(C.byref(desc)))
+
+
 def sv_accept(desc: SvAcceptDesc, target_logits, draft_probs, draft_tokens, temperature: float,
               philox_seed: int, accept_len, next_token, accept_path=None, status_flags=None,
-              stream=None) -> None:
+              workspace=None, workspace_bytes: int = 0, stream=None) -> None:
     _check(_L().sv_accept(C.byref(desc), _ptr(target_logits), _ptr(draft_probs), _ptr(draft_tokens),
                           float(temperature), int(philox_seed) & 0xFFFFFFFFFFFFFFFF, _ptr(accept_len),
-                          _ptr(next_token), _ptr(accept_path), _ptr(status_flags), _stream(stream)))
+                          _ptr(next_token), _ptr(accept_path), _ptr(status_flags), _ptr(workspace),
+                          int(workspace_bytes), _stream(stream)))
 
 
 def sv_kv_commit(desc: SvAttnDesc, layers, block_table, ctx_lens, accept_len, accept_path, new_ctx_lens,

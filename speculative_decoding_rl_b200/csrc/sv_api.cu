@@ -221,26 +221,52 @@ sv_status sv_cascade_verify_attention(const sv_attn_desc *d, const sv_cascade_de
     return SV_OK;
 }
 
-sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const float *draft_probs,
-                    const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
-                    int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
-                    int32_t *status_flags, void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks every argument of sv_accept that the workspace size depends on; fills p.
+sv_status check_accept_desc(const sv_accept_desc *d, float temperature, sv::AcceptParams *p) {
     if (!d) return fail(SV_ERR_INVALID_ARG, "desc is NULL");
     if (d->num_seqs < 0) return fail(SV_ERR_INVALID_ARG, "num_seqs < 0");
     if (d->num_rows < 1 || d->num_rows > 64) return fail(SV_ERR_INVALID_ARG, "num_rows must be in [1, 64]");
     if (d->vocab < 1) return fail(SV_ERR_INVALID_ARG, "vocab < 1");
-    if (d->vocab > sv::accept_max_vocab()) return fail(SV_ERR_UNSUPPORTED, "vocab above %d", sv::accept_max_vocab());
+    if (d->vocab > sv::ACC_MAX_VOCAB) return fail(SV_ERR_UNSUPPORTED, "vocab above %d", sv::ACC_MAX_VOCAB);
     if (d->num_seqs > 65535) return fail(SV_ERR_UNSUPPORTED, "num_seqs above 65535");
     if (!(temperature >= 0.f) || isinf(temperature)) return fail(SV_ERR_INVALID_ARG, "temperature must be finite and >= 0");
-    const bool greedy = temperature == 0.f;
-    sv::AcceptParams p = {};
-    p.parent[0] = -1;
+    *p = sv::AcceptParams{};
+    p->parent[0] = -1;
     for (int c = 1; c < d->num_rows; ++c) {
         const int par = d->tree_parents ? d->tree_parents[c] : c - 1;
         if (par < 0 || par >= c) return fail(SV_ERR_INVALID_ARG, "tree_parents[%d] = %d is not in [0, %d)", c, par, c);
-        p.parent[c] = (int8_t)par;
+        p->parent[c] = (int8_t)par;
     }
     if (d->tree_parents && d->tree_parents[0] != -1) return fail(SV_ERR_INVALID_ARG, "tree_parents[0] must be -1");
+    p->B = d->num_seqs;
+    p->N = d->num_rows;
+    p->V = d->vocab;
+    p->S = (d->vocab + sv::ACC_SLICE - 1) / sv::ACC_SLICE;
+    return SV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sv_accept_workspace_size(const sv_accept_desc *d) {
+    sv::AcceptParams p;
+    if (check_accept_desc(d, 1.f, &p) != SV_OK) return 0;
+    return sv::accept_workspace_bytes(p.B, p.N, p.V);
+}
+
+sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const float *draft_probs,
+                    const int32_t *draft_tokens, float temperature, uint64_t philox_seed,
+                    int32_t *accept_len, int32_t *next_token, int32_t *accept_path,
+                    int32_t *status_flags, void *workspace, size_t workspace_bytes, void *stream) {
+    sv::AcceptParams p;
+    sv_status s = check_accept_desc(d, temperature, &p);
+    if (s != SV_OK) return s;
+    const bool greedy = temperature == 0.f;
     if (d->num_seqs == 0) return SV_OK;
     if (!target_logits || !accept_len || !next_token) return fail(SV_ERR_INVALID_ARG, "a required pointer is NULL");
     if (d->num_rows > 1 && !draft_tokens) return fail(SV_ERR_INVALID_ARG, "draft_tokens is NULL");
@@ -249,6 +275,9 @@ sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const f
         (draft_tokens && !aligned(draft_tokens, 4)) || !aligned(accept_len, 4) || !aligned(next_token, 4) ||
         (accept_path && !aligned(accept_path, 4)) || (status_flags && !aligned(status_flags, 4)))
         return fail(SV_ERR_INVALID_ARG, "misaligned pointer");
+    const size_t need = sv::accept_workspace_bytes(p.B, p.N, p.V);
+    if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
+        return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);
     p.logits = target_logits;
     p.q = draft_probs;
     p.drafts = draft_tokens;
@@ -256,14 +285,13 @@ sv_status sv_accept(const sv_accept_desc *d, const float *target_logits, const f
     p.next_token = next_token;
     p.accept_path = accept_path;
     p.status = status_flags;
-    p.B = d->num_seqs;
-    p.N = d->num_rows;
-    p.V = d->vocab;
     p.greedy = greedy ? 1 : 0;
     p.log2e_over_T = greedy ? 0.f : (float)(1.4426950408889634 / (double)temperature);
     p.key.k0 = (uint32_t)(philox_seed & 0xFFFFFFFFull);
     p.key.k1 = (uint32_t)(philox_seed >> 32);
-    cudaError_t e = sv::launch_accept(p, static_cast<cudaStream_t>(stream));
+    p.workspace = workspace;
+    const int rounds = greedy ? 0 : sv::accept_rounds(p.parent, p.N);
+    cudaError_t e = sv::launch_accept(p, rounds, static_cast<cudaStream_t>(stream), nullptr);
     if (e != cudaSuccess) return fail(SV_ERR_CUDA, "accept launch: %s", cudaGetErrorString(e));
     return SV_OK;
 }

@@ -559,8 +559,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const int tpre = ups * TP[fb] + fhr * Tb;
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
-            // a cascade call merges every unit with its shared prefix: always a slot
-            const bool to_slot = nseg > 1 || p.pp_o != nullptr;
+            const bool to_slot = nseg > 1;
             float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
             // O^T in chunks of 16 columns (few live registers)
 #pragma unroll 1
@@ -574,11 +573,26 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     for (int c = 0; c < 16; ++c) {
                         const int r = col0 + c0 + c;
                         if (r < frows) {
-                            const float l = lfin[r];
-                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
+                            float l = lfin[r], num = o[c];
                             const int ridx = frc * p.rows_unit + r;
                             const int i = ridx / p.G, hq = fh * p.G + (ridx - i * p.G);
-                            p.out[(((size_t)fb * p.N + i) * p.Hq + hq) * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
+                            const size_t orow = ((size_t)fb * p.N + i) * p.Hq + hq;
+                            if (p.pp_o) {
+                                // cascade call: merge the row's shared-prefix partials by log-sum-exp
+                                const size_t pstride = (size_t)p.B * p.N * p.Hq;
+                                float m = mfin[r];
+                                for (int sp = 0; sp < p.pp_splits; ++sp) {
+                                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.pp_ml) + sp * pstride + orow);
+                                    const float op = __ldcg(p.pp_o + (sp * pstride + orow) * D + ell);
+                                    const float M = fmaxf(m, ml.x);
+                                    const float a = ex2_approx(m - M), bq = ex2_approx(ml.x - M);
+                                    num = num * a + op * bq;
+                                    l = l * a + ml.y * bq;
+                                    m = M;
+                                }
+                            }
+                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? num / l : 0.f);
+                            p.out[orow * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
                         }
                     }
                 } else {
@@ -812,8 +826,9 @@ SV_DEV int block_sum_i(int v, int *red) {
 // sequence by its status warp). One CTA per (COMBINE_ROWS rows, unit), one warp
 // per row, four head dimensions per lane:
 //   M = max_k m_k,  L = sum_k 2^(m_k - M) l_k,  out = sum_k 2^(m_k - M) O_k / L.
-// In a cascade call every unit has slots and the shared prefix's partials of
-// the row join the merge as further terms k.
+// In a cascade call the shared prefix's partials of the row join the merge of
+// a split unit as further terms k (a whole unit merged them in the attention
+// kernel).
 // Launched as a programmatic dependent of the attention kernel, which lets it
 // launch only after its own wait on earlier work: the schedule is recomputed
 // from ctx_lens (complete by then) before this kernel waits, so once the
@@ -849,7 +864,7 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     const int W = (total + p.num_ctas - 1) / p.num_ctas;
     const int tpre = ups * before + hr * Tb;
     const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
-    if (n == 1 && !p.pp_o) return;
+    if (n == 1) return;  // written by the attention kernel (a cascade call's prefix merged there too)
     const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const size_t sf = slot_stride(RU, D);
@@ -968,8 +983,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Pool map: boxes of 16 keys x 64 dims, 128B-swizzled, for the shared-memory
 // tiles; with whole_page, 16 keys x D dims un-swizzled, for L2 prefetches.
-static bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D,
-                            bool whole_page = false) {
+bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D, bool whole_page) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)PAGE, (cuuint64_t)Hkv, (cuuint64_t)num_blocks};

@@ -1,6 +1,7 @@
 // Internal declarations shared by the libspecverify translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -10,9 +11,10 @@
 namespace sv {
 
 // ----------------------------- accept ---------------------------------------
-constexpr int ACC_MAX_CHUNK_FLOATS = 55 * 1024;  // per-CTA vocabulary slice held in shared memory
-
-struct PhiloxKeyHost { uint32_t k0, k1; };
+// The vocabulary is cut into slices of ACC_SLICE entries; every pass over a
+// row is one CTA per (row, slice).
+constexpr int ACC_SLICE = 8192;
+constexpr int ACC_MAX_VOCAB = 1 << 22;
 
 struct AcceptParams {
     const float *logits;
@@ -22,15 +24,22 @@ struct AcceptParams {
     int32_t *next_token;
     int32_t *accept_path;
     int32_t *status;
-    int B, N, V, chunk;
-    float log2e_over_T;   // log2(e) / T for T > 0
+    int B, N, V, S;        // S = slices per row
+    float log2e_over_T;    // log2(e) / T for T > 0
     int greedy;
     struct { uint32_t k0, k1; } key;
     int8_t parent[64];
+    void *workspace;       // accept_workspace_bytes(B, N, V), 256-byte aligned
 };
 
-int accept_max_vocab();
-cudaError_t launch_accept(const AcceptParams &p, cudaStream_t stream);
+size_t accept_workspace_bytes(int B, int N, int V);
+// Passes over rejected rows (each a pass kernel and a walk kernel) the walk
+// can need for this tree: the largest number of rejections on the way to a
+// node, plus that node's children (one pass for a node without children).
+int accept_rounds(const int8_t *parent, int N);
+// Launches the whole accept (stats, walk, then `rounds` pass + walk pairs;
+// greedy: stats and walk only). Returns the number of kernels launched in *launches.
+cudaError_t launch_accept(const AcceptParams &p, int rounds, cudaStream_t stream, int *launches);
 
 // ----------------------------- attention ------------------------------------
 // Keys per work tile: the split-context schedule hands out tiles of TILE_KEYS
@@ -68,6 +77,10 @@ struct AttnParams {
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
+// TMA map of a K or V pool [num_blocks][Hkv][16][D]: boxes of 16 keys x 64 dims,
+// 128-byte swizzled (whole_page: 16 keys x D, unswizzled). A block id of
+// num_blocks addresses past the pool and loads zeros.
+bool encode_pool_map(CUtensorMap *m, const void *pool, int num_blocks, int Hkv, int D, bool whole_page = false);
 // Row chunks of a unit: rows_unit rows (i, g) per chunk, RC chunks, Nc whole query rows i per chunk.
 void row_chunks(int N, int G, int *rows_unit, int *RC, int *Nc);
 int attention_num_ctas();
@@ -75,9 +88,9 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
 
 // ------------------------------ cascade ------------------------------------
 // Shared-prefix pass: one CTA of CASCADE_ROWS query rows per (group, KV head,
-// row chunk, prefix split).
-constexpr int CASCADE_ROWS = 64;
-constexpr int CASCADE_KEYS = 64;
+// row tile, prefix split), CASCADE_KEYS keys per tile.
+constexpr int CASCADE_ROWS = 128;
+constexpr int CASCADE_KEYS = 128;
 
 struct CascadePlan {
     int num_groups, splits, items;

@@ -12,8 +12,8 @@ from typing import Optional
 import torch
 
 from . import (SvAttnDesc, SvPagedKV, make_accept_desc, make_cascade_desc, make_kv_layers, sv_accept,
-               sv_cascade_attention_workspace_size, sv_cascade_verify_attention, sv_kv_commit,
-               sv_verify_attention, sv_verify_attention_workspace_size)
+               sv_accept_workspace_size, sv_cascade_attention_workspace_size, sv_cascade_verify_attention,
+               sv_kv_commit, sv_verify_attention, sv_verify_attention_workspace_size)
 
 
 class AttentionCall:
@@ -83,11 +83,14 @@ class AcceptCall:
         self.next_token = torch.full((B,), -7, dtype=torch.int32, device=dev)
         self.path = torch.full((B, max(N - 1, 1)), -7, dtype=torch.int32, device=dev) if with_path else None
         self.status = torch.full((B,), -7, dtype=torch.int32, device=dev) if with_status else None
+        self.ws_bytes = sv_accept_workspace_size(self.desc)
+        self.workspace = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=dev)
 
     def run(self, stream=None):
         sv_accept(self.desc, self.logits, self.q if self.q.numel() else None,
                   self.drafts if self.drafts.numel() else None, self.temperature, self.seed,
-                  self.accept_len, self.next_token, self.path, self.status, stream)
+                  self.accept_len, self.next_token, self.path, self.status, self.workspace, self.ws_bytes,
+                  stream)
         return self.accept_len, self.next_token
 
 

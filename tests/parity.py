@@ -78,3 +78,30 @@ def compare_accept(gpu_len, gpu_next, gpu_path, gpu_status, orc, greedy: bool):
         if gpu_next[b] != orc.next_token[b]:
             bad.append((b, f"next_token {int(gpu_next[b])} != {int(orc.next_token[b])}"))
     return bad, exempt
+
+
+def host_threads() -> int:
+    import os
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def all_rows(a) -> np.ndarray:
+    """Every (b, i, hq) output row of an attention input set."""
+    b, i, h = np.meshgrid(np.arange(a.num_seqs), np.arange(a.num_q_rows), np.arange(a.num_q_heads), indexing="ij")
+    return np.stack([b.ravel(), i.ravel(), h.ravel()], axis=1).astype(np.int32)
+
+
+def oracle_rows_parallel(a, rows: np.ndarray, threads: int = 0) -> np.ndarray:
+    """oracle.attention_rows over chunks of rows on several host threads (the
+    oracle is reentrant C and its binding releases the GIL); same values as one
+    call, in the order of ``rows``."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    threads = threads or host_threads()
+    chunks = np.array_split(rows, max(1, min(4 * threads, len(rows))))
+    with ThreadPoolExecutor(threads) as ex:
+        parts = list(ex.map(lambda r: oracle.attention_rows(a, r), chunks))
+    return np.concatenate(parts) if parts else np.zeros((0, a.head_dim))

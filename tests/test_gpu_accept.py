@@ -27,30 +27,95 @@ def run_both(a, seed, temperature=None):
     return bad, exempt, orc, call
 
 
+# Near-tie exemptions are bounded, not just counted. An accept test is a near
+# tie when |u - r(d)/q(d)| < 1e-5, which a uniform u hits with probability
+# about 2e-5 per test: more than 1% of sequences would mean the comparison is
+# broken. A draw is a near tie when its threshold falls within 1e-5 of the
+# mass of a CDF step; with a vocabulary of ~1.5e5 tokens the smaller steps are
+# themselves below 1e-5, so a sizeable share of draws qualifies (about 15-20%
+# at the full-size configurations); every exempt draw must still land in the
+# oracle's band of tokens reachable by thresholds within 1e-5.
+MAX_TIE_TEST_SHARE = 0.01
+MAX_TIE_DRAW_SHARE = 0.40
+
+
+def check_exemptions(orc, what):
+    n = len(orc.accept_len)
+    ties = int((orc.tie_depth >= 0).sum())
+    draws = int(((orc.tie_depth < 0) & (orc.tie_draw > 0)).sum())
+    print(f"{what}: {n} sequences, {ties} accept-test near ties, {draws} near-tie draws")
+    assert ties <= max(1, MAX_TIE_TEST_SHARE * n), (what, ties)
+    assert draws <= max(2, MAX_TIE_DRAW_SHARE * n), (what, draws)
+    return ties + draws
+
+
 @pytest.mark.parametrize("name,over,T", [
     ("tiny_chain", {}, 1.0),
     ("tiny_chain", {}, 0.0),
     ("qwen7b_longtail", {}, 1.0),
-    ("qwen32b_sweep", dict(num_seqs=16, gamma=8), 1.0),
-    ("qwen32b_sweep", dict(num_seqs=4, gamma=2), 1.0),
+    ("qwen7b_longtail", {}, 0.0),
     ("tree_qwen3_30b", {}, 1.0),
+    ("tree_qwen3_30b", {}, 0.0),
     ("grpo_shared_prefix", dict(temperature=0.0), 0.0),
     ("grpo_shared_prefix", dict(temperature=0.7), 0.7),
 ])
 def test_accept_matches_oracle(name, over, T):
     w = W.workload(name, **over)
     a = W.build_accept(w)
-    total_exempt = 0
     for seed in (0, 1, 12345678901):
         bad, exempt, orc, _ = run_both(a, seed, T)
         assert not bad, f"{name} seed {seed}: {bad[:5]}"
-        total_exempt += exempt
-    print(f"{name} T={T}: {a.num_seqs * 3} sequences, {total_exempt} near-tie exemptions")
+        check_exemptions(orc, f"{name} T={T} seed {seed}")
+
+
+# every point of the Qwen2.5-32B batch-shrink sweep at full vocabulary, every sequence
+@pytest.mark.parametrize("B", [256, 64, 16, 4, 1])
+@pytest.mark.parametrize("gamma", [2, 4, 8])
+def test_accept_32b_sweep_every_point(B, gamma):
+    a = W.build_accept(W.workload("qwen32b_sweep", num_seqs=B, gamma=gamma))
+    for seed in (0, 7):
+        bad, exempt, orc, _ = run_both(a, seed)
+        assert not bad, f"B={B} gamma={gamma} seed {seed}: {bad[:5]}"
+        check_exemptions(orc, f"32B sweep B={B} gamma={gamma} seed {seed}")
+    bad, _, _, _ = run_both(a, 3, temperature=0.0)
+    assert not bad, f"B={B} gamma={gamma} greedy: {bad[:5]}"
+
+
+def test_accept_workspace_needs_no_initialisation():
+    # the workspace is written before it is read: garbage in it changes nothing
+    a = W.build_accept(W.workload("tree_qwen3_30b"))
+    ref = AcceptCall(a, seed=5)
+    ref.run()
+    for fill in (0xFF, 0x7F, 0x00):
+        c = AcceptCall(a, seed=5)
+        c.workspace.fill_(fill)
+        c.run()
+        torch.cuda.synchronize()
+        for x, y in ((c.accept_len, ref.accept_len), (c.next_token, ref.next_token), (c.path, ref.path),
+                     (c.status, ref.status)):
+            assert torch.equal(x, y)
+
+
+def test_accept_back_to_back_calls_share_nothing():
+    # two calls with their own workspaces on one stream, then the same two reversed
+    a1 = W.build_accept(W.workload("qwen32b_sweep", num_seqs=16, gamma=4))
+    a2 = W.build_accept(W.workload("tree_qwen3_30b"))
+    c1, c2 = AcceptCall(a1, seed=1), AcceptCall(a2, seed=2)
+    c1.run(); c2.run()
+    torch.cuda.synchronize()
+    r1 = [t.clone() for t in (c1.accept_len, c1.next_token)]
+    r2 = [t.clone() for t in (c2.accept_len, c2.next_token)]
+    c2.run(); c1.run()
+    torch.cuda.synchronize()
+    assert torch.equal(r1[0], c1.accept_len) and torch.equal(r1[1], c1.next_token)
+    assert torch.equal(r2[0], c2.accept_len) and torch.equal(r2[1], c2.next_token)
 
 
 def test_accept_many_small_problems():
-    # many sequences, small vocab, chain and tree, several seeds
-    for parents in (None, W.TREE_PARENTS_3221, [-1, 0, 0, 1, 1, 2]):
+    # many sequences, small vocab, chain and trees (wide fan-outs: many rejections
+    # in a row at one node, each a pass of its own), several seeds
+    for parents in (None, W.TREE_PARENTS_3221, [-1, 0, 0, 1, 1, 2], [-1, 0, 0, 0, 0, 0, 0, 0],
+                    [-1, 0, 0, 0, 1, 1, 1, 2, 2, 3, 4, 4, 4]):
         N = 5 if parents is None else len(parents)
         a = W.make_accept_inputs(512, N, 37, seed=9, logit_std=1.0, draft_noise=0.8, temperature=1.0,
                                  parents=parents)
@@ -62,7 +127,9 @@ def test_accept_many_small_problems():
 
 
 def test_accept_gamma_zero_and_vocab_edges():
-    for V in (1, 3, 8, 1001, 4099):
+    # vocabularies around the 8192-entry slice (one slice, a ragged last slice,
+    # exactly two slices, not a multiple of 4: scalar loads)
+    for V in (1, 3, 8, 1001, 4099, 8191, 8192, 8193, 16384, 20001):
         a = W.make_accept_inputs(64, 1, V, seed=V, logit_std=2.0, draft_noise=0.5, temperature=1.0)
         bad, _, _, _ = run_both(a, 7)
         assert not bad, (V, bad[:5])

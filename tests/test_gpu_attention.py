@@ -1,16 +1,19 @@
 """GPU parity of sv_verify_attention against the fp64 oracle (B200).
 
 Full-output comparison at sizes the oracle finishes in seconds (several tiles,
-ragged tails, all five workload shapes), sampled-row comparison at the bench's
-full size, and edge cases: single key, tile-boundary lengths, >128 query rows
-per KV head, explicit vs implicit chain masks, invalid contexts and block ids.
+ragged tails, all five workload shapes); at full size, every output row of the
+7B long-tail and the tree layers, every point of the 32B batch-shrink sweep
+(all rows up to 4 sequences, else sampled rows plus the longest sequence) and
+sampled rows of the GRPO group; and edge cases: single key, tile-boundary
+lengths, >128 query rows per KV head, explicit vs implicit chain masks,
+invalid contexts and block ids.
 """
 import numpy as np
 import pytest
 import torch
 
 import oracle
-from parity import assert_attention_close
+from parity import all_rows, assert_attention_close, oracle_rows_parallel
 from speculative_decoding_rl_b200 import workloads as W
 from speculative_decoding_rl_b200.session import AttentionCall
 
@@ -102,34 +105,6 @@ def test_attention_flags_invalid_sequences():
     assert_attention_close(got[3], want[3], "valid sequence next to invalid ones")
 
 
-def test_attention_full_size_sampled_rows():
-    # The bench workload at full size; the oracle computes a seeded sample of rows.
-    w = W.workload("qwen7b_longtail")
-    a = W.build_attention(w)
-    got, st = run(a)
-    assert (st == 0).all()
-    rng = np.random.default_rng(0)
-    rows = np.stack([rng.integers(0, a.num_seqs, 96), rng.integers(0, a.num_q_rows, 96),
-                     rng.integers(0, a.num_q_heads, 96)], axis=1).astype(np.int32)
-    want = oracle.attention_rows(a, rows)
-    sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
-    max_abs, mean_rel = assert_attention_close(sel, want, "qwen7b full size, sampled rows")
-    print(f"full-size sampled: max_abs {max_abs:.2e} mean_rel {mean_rel:.2e}")
-
-
-def test_tree_full_size_sampled_rows():
-    w = W.workload("tree_qwen3_30b")
-    a = W.build_attention(w)
-    got, st = run(a)
-    assert (st == 0).all()
-    rng = np.random.default_rng(1)
-    rows = np.stack([rng.integers(0, a.num_seqs, 48), rng.integers(0, a.num_q_rows, 48),
-                     rng.integers(0, a.num_q_heads, 48)], axis=1).astype(np.int32)
-    want = oracle.attention_rows(a, rows)
-    sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
-    assert_attention_close(sel, want, "tree full size, sampled rows")
-
-
 def test_split_units_need_no_workspace_initialisation():
     # A 40k-token sequence next to a short one: its units are split over dozens
     # of CTAs and merged by the last to arrive. The workspace starts as random
@@ -153,13 +128,11 @@ def test_split_units_need_no_workspace_initialisation():
 
 
 @pytest.mark.parametrize("name,over,nrows", [
-    ("qwen32b_sweep", dict(num_seqs=64, gamma=8), 64),
-    ("qwen32b_sweep", dict(num_seqs=256, gamma=2), 48),
-    ("grpo_shared_prefix", {}, 64),
+    ("grpo_shared_prefix", {}, 256),
 ])
 def test_full_size_sampled_rows_other_shapes(name, over, nrows):
-    # the 32B-shaped sweep points (64 and 256 sequences) and the GRPO group with
-    # its shared prompt pages, at full size; the oracle computes sampled rows
+    # the GRPO group with its shared prompt pages, at full size; the oracle
+    # computes sampled rows
     w = W.workload(name, **over)
     a = W.build_attention(w)
     got, st = run(a)
@@ -167,6 +140,42 @@ def test_full_size_sampled_rows_other_shapes(name, over, nrows):
     rng = np.random.default_rng(sum(map(ord, name)) + len(over))
     rows = np.stack([rng.integers(0, a.num_seqs, nrows), rng.integers(0, a.num_q_rows, nrows),
                      rng.integers(0, a.num_q_heads, nrows)], axis=1).astype(np.int32)
-    want = oracle.attention_rows(a, rows)
+    want = oracle_rows_parallel(a, rows)
     sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
     assert_attention_close(sel, want, f"{name} {over} full size, sampled rows")
+
+
+@pytest.mark.parametrize("name", ["qwen7b_longtail", "tree_qwen3_30b"])
+def test_full_size_full_output(name):
+    # every output row of the full-size layer against the oracle (rows spread over host threads)
+    a = W.build_attention(W.workload(name))
+    got, st = run(a)
+    assert (st == 0).all()
+    rows = all_rows(a)
+    want = oracle_rows_parallel(a, rows)
+    max_abs, mean_rel = assert_attention_close(got[rows[:, 0], rows[:, 1], rows[:, 2]], want,
+                                               f"{name} full size, every row")
+    print(f"{name} full output ({len(rows)} rows): max_abs {max_abs:.2e} mean_rel {mean_rel:.2e}")
+
+
+@pytest.mark.parametrize("B", [256, 64, 16, 4, 1])
+@pytest.mark.parametrize("gamma", [2, 4, 8])
+def test_32b_sweep_every_point(B, gamma):
+    # each point of the Qwen2.5-32B batch-shrink sweep at full size: every row
+    # up to 4 sequences, else 64 seeded rows plus every row of the longest sequence
+    a = W.build_attention(W.workload("qwen32b_sweep", num_seqs=B, gamma=gamma))
+    got, st = run(a)
+    assert (st == 0).all()
+    if B <= 4:
+        rows = all_rows(a)
+    else:
+        rng = np.random.default_rng(1000 * B + gamma)
+        samp = np.stack([rng.integers(0, B, 64), rng.integers(0, a.num_q_rows, 64),
+                         rng.integers(0, a.num_q_heads, 64)], axis=1).astype(np.int32)
+        longest = int(np.argmax(a.ctx_lens.numpy()))
+        whole = all_rows(a)
+        rows = np.concatenate([samp, whole[whole[:, 0] == longest]])
+    want = oracle_rows_parallel(a, rows)
+    max_abs, mean_rel = assert_attention_close(got[rows[:, 0], rows[:, 1], rows[:, 2]], want,
+                                               f"32B sweep B={B} gamma={gamma}")
+    print(f"32B sweep B={B} gamma={gamma} ({len(rows)} rows): max_abs {max_abs:.2e} mean_rel {mean_rel:.2e}")

@@ -22,7 +22,7 @@ def declared_functions():
 
 def test_header_declares_the_entry_points():
     names = declared_functions()
-    for n in ("sv_verify_attention", "sv_verify_attention_workspace_size", "sv_accept",
+    for n in ("sv_verify_attention", "sv_verify_attention_workspace_size", "sv_accept", "sv_accept_workspace_size",
               "sv_testing_philox4x32_10", "sv_testing_verify_attention_stalled",
               "sv_cascade_verify_attention", "sv_cascade_attention_workspace_size",
               "sv_status_string", "sv_last_error", "sv_version"):
@@ -160,6 +160,21 @@ def test_accept_rejects_bad_arguments(kw, parents, temp, status):
     with pytest.raises(sv.SvError) as e:
         sv.sv_accept(desc, 16, 16, 16, temp, 0, 16, 16, None, None, stream=0)
     assert e.value.status == status
+
+
+def test_accept_workspace_is_required_and_sized():
+    desc = sv.make_accept_desc(4, 5, 1000)
+    need = sv.sv_accept_workspace_size(desc)
+    assert need > 0 and need % 256 == 0
+    assert sv.sv_accept_workspace_size(sv.make_accept_desc(8, 5, 1000)) > need
+    assert sv.sv_accept_workspace_size(sv.make_accept_desc(4, 5, 100_000)) > need
+    assert sv.sv_accept_workspace_size(sv.make_accept_desc(4, 0, 1000)) == 0
+    assert sv.sv_accept_workspace_size(sv.make_accept_desc(4, 5, 10_000_000)) == 0
+    for ws, nbytes in [(None, need), (256, need - 1), (128, need)]:
+        with pytest.raises(sv.SvError) as e:
+            sv.sv_accept(desc, 16, 16, 16, 1.0, 0, 16, 16, None, None, ws, nbytes, stream=0)
+        assert e.value.status == sv.SV_ERR_WORKSPACE
+        assert "workspace" in sv.sv_last_error()
 
 
 def test_accept_requires_outputs_and_drafts():
