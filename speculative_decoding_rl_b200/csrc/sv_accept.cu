@@ -259,20 +259,26 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_pass_kernel(const AcceptPa
     const float M = s_M, Sv = s_S, c = p.log2e_over_T;
     float wsum = 0.f, psum = 0.f;
     if (VEC && k <= 1) {
-        // p alone, or the chain case (one draft row): 16-byte loads
+        // p alone, or the chain case (one draft row): 16-byte loads, all of a
+        // thread's loads in flight before the first is used
         const float4 *l4 = reinterpret_cast<const float4 *>(lrow);
         const float4 *q4 = reinterpret_cast<const float4 *>(k ? s_q[0] : lrow);
-#pragma unroll 2
-        for (int i = tid; 4 * i < n; i += ACC_THREADS) {
-            const float4 lv = __ldg(l4 + i);
-            const float e0 = exp2f((lv.x - M) * c), e1 = exp2f((lv.y - M) * c);
-            const float e2 = exp2f((lv.z - M) * c), e3 = exp2f((lv.w - M) * c);
+        constexpr int J = ACC_PER_THREAD / 4;
+        float4 lv[J], qv[J];
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const int i = tid + j * ACC_THREADS;
+            lv[j] = 4 * i < n ? __ldg(l4 + i) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+            qv[j] = (k && 4 * i < n) ? __ldg(q4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < J; ++j) {
+            const float e0 = exp2f((lv[j].x - M) * c), e1 = exp2f((lv[j].y - M) * c);
+            const float e2 = exp2f((lv[j].z - M) * c), e3 = exp2f((lv[j].w - M) * c);
             psum += (e0 + e1) + (e2 + e3);
-            if (k) {
-                const float4 qv = __ldg(q4 + i);
-                wsum += (fmaxf(e0 / Sv - qv.x, 0.f) + fmaxf(e1 / Sv - qv.y, 0.f)) +
-                        (fmaxf(e2 / Sv - qv.z, 0.f) + fmaxf(e3 / Sv - qv.w, 0.f));
-            }
+            if (k)
+                wsum += (fmaxf(e0 / Sv - qv[j].x, 0.f) + fmaxf(e1 / Sv - qv[j].y, 0.f)) +
+                        (fmaxf(e2 / Sv - qv[j].z, 0.f) + fmaxf(e3 / Sv - qv[j].w, 0.f));
         }
     } else {
         for (int x = tid; x < n; x += ACC_THREADS) {
@@ -351,7 +357,9 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
     const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const AccPtrs W = acc_ptrs(p);
     __shared__ AccState S;
-    __shared__ float wbuf[ACC_SLICE];  // draw: the weights of the drawn slice
+    // draw: the weights of the drawn slice, one pad word after every 32 so that
+    // a thread's contiguous segment of 32 sits in 32 different banks
+    __shared__ float wbuf[ACC_SLICE + ACC_SLICE / 32];
     __shared__ float2 rs[ACC_MAX_VOCAB / ACC_SLICE];  // the pass's per-slice sums
     __shared__ int s_action, s_nonfinite, s_owner, s_first;
     __shared__ float s_t;
@@ -491,19 +499,49 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
     const int x0 = s_owner * ACC_SLICE;
     const int n = min(ACC_SLICE, p.V - x0);
     {
-        // the drawn slice's weights, with the pass's arithmetic, staged in shared memory
+        // the drawn slice's weights, with the pass's arithmetic, staged in shared
+        // memory; a thread's loads are all in flight before the first is used
         const float *lrow = p.logits + ((size_t)b * N + v) * p.V + x0;
         const float M = S.rowM[v], Sv = S.rowS[v];
-        for (int x = tid; x < n; x += WALK_THREADS) {
-            const float e = exp2f((__ldg(lrow + x) - M) * c);
-            float wgt = e;
-            if (use_w) {
-                float r = e / Sv;
-                for (int i = 0; i + 1 < k; ++i)
-                    r = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[i] - 1) * p.V + x0 + x), 0.f) / S.Z[i];
-                wgt = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[k - 1] - 1) * p.V + x0 + x), 0.f);
+        auto put = [&](int x, float wgt) { wbuf[x + (x >> 5)] = wgt; };
+        if (p.vec && k <= 1) {
+            const float4 *l4 = reinterpret_cast<const float4 *>(lrow);
+            const float4 *q4 = k ? reinterpret_cast<const float4 *>(
+                                       p.q + ((size_t)b * (N - 1) + S.chain[0] - 1) * p.V + x0)
+                                 : l4;
+            constexpr int J = ACC_SLICE / (4 * WALK_THREADS);
+            float4 lv[J], qv[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int i = tid + j * WALK_THREADS;
+                lv[j] = 4 * i < n ? __ldg(l4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+                qv[j] = (k && 4 * i < n) ? __ldg(q4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
             }
-            wbuf[x] = wgt;
+#pragma unroll
+            for (int j = 0; j < J; ++j) {
+                const int i = tid + j * WALK_THREADS;
+                if (4 * i >= n) continue;
+                const float l[4] = {lv[j].x, lv[j].y, lv[j].z, lv[j].w};
+                const float q[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float ex = exp2f((l[e] - M) * c);
+                    put(4 * i + e, k ? fmaxf(ex / Sv - q[e], 0.f) : ex);
+                }
+            }
+        } else {
+            for (int x = tid; x < n; x += WALK_THREADS) {
+                const float e = exp2f((__ldg(lrow + x) - M) * c);
+                float wgt = e;
+                if (use_w) {
+                    float r = e / Sv;
+                    for (int i = 0; i + 1 < k; ++i)
+                        r = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[i] - 1) * p.V + x0 + x), 0.f) /
+                            S.Z[i];
+                    wgt = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[k - 1] - 1) * p.V + x0 + x), 0.f);
+                }
+                put(x, wgt);
+            }
         }
     }
     __syncthreads();
@@ -513,7 +551,7 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
     float tsum = 0.f;
     int tlast = -1;
     for (int x = s0; x < s1; ++x) {
-        const float wv = wbuf[x];
+        const float wv = wbuf[x + (x >> 5)];
         tsum += wv;
         if (wv > 0.f) tlast = x;
     }
@@ -555,8 +593,9 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
         float cl = 0.f;
         tok = x0 + max(tlast, s0);
         for (int x = s0; x < s1; ++x) {
-            cl += wbuf[x];
-            if (wbuf[x] > 0.f && cl > tj) { tok = x0 + x; break; }
+            const float wv = wbuf[x + (x >> 5)];
+            cl += wv;
+            if (wv > 0.f && cl > tj) { tok = x0 + x; break; }
         }
     }
     if (tok >= 0) {
@@ -596,9 +635,12 @@ static cudaError_t launch_pdl(void (*kfn)(Args...), dim3 grid, dim3 block, cudaS
     return cudaLaunchKernelEx(&cfg, kfn, args...);
 }
 
-cudaError_t launch_accept(const AcceptParams &p, int rounds, cudaStream_t stream, int *launches) {
+cudaError_t launch_accept(const AcceptParams &p0, int rounds, cudaStream_t stream, int *launches) {
     auto a16 = [](const void *x) { return (reinterpret_cast<uintptr_t>(x) & 15) == 0; };
-    const bool vec = (p.V % 4 == 0) && a16(p.logits) && (p.greedy || p.q == nullptr || a16(p.q));
+    const bool vec = (p0.V % 4 == 0) && a16(p0.logits) && (p0.greedy || p0.q == nullptr || a16(p0.q));
+    AcceptParams pv = p0;
+    pv.vec = vec ? 1 : 0;
+    const AcceptParams &p = pv;
     const dim3 sgrid((unsigned)p.S, (unsigned)p.N, (unsigned)p.B);
     cudaError_t e;
     int n = 0;

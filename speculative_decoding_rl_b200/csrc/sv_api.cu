@@ -109,6 +109,7 @@ sv::AttnParams attn_params(const sv_attn_desc *d, const void *q, const sv_paged_
     p.ws_partial = static_cast<float *>(workspace);
     p.wait_limit_ns = 2000000000ull;
     p.stall = 0;
+    p.all_slots = 0;
     return p;
 }
 
@@ -188,10 +189,8 @@ size_t sv_cascade_attention_workspace_size(const sv_attn_desc *d, const sv_casca
     if (check_attn_desc(d) != SV_OK || check_cascade_desc(d, c) != SV_OK) return 0;
     const int ctas = sv::attention_num_ctas();
     if (ctas <= 0) return 0;
-    sv::CascadePlan plan;
-    sv::cascade_plan(c, d->num_q_rows, d->num_q_heads, d->num_kv_heads, ctas, &plan);
     return sv::cascade_workspace(d->num_seqs, d->num_q_rows, d->num_q_heads, d->num_kv_heads, d->head_dim,
-                                 d->max_blocks_per_seq, ctas, plan.splits)
+                                 d->max_blocks_per_seq, ctas)
         .total;
 }
 
@@ -208,9 +207,9 @@ sv_status sv_cascade_verify_attention(const sv_attn_desc *d, const sv_cascade_de
     const int ctas = sv::attention_num_ctas();
     if (ctas <= 0) return fail(SV_ERR_CUDA, "cannot query the current device");
     sv::CascadePlan plan;
-    sv::cascade_plan(c, d->num_q_rows, d->num_q_heads, d->num_kv_heads, ctas, &plan);
+    sv::cascade_plan(c, d->num_q_rows, d->num_q_heads, d->num_kv_heads, &plan);
     const size_t need = sv::cascade_workspace(d->num_seqs, d->num_q_rows, d->num_q_heads, d->num_kv_heads,
-                                              d->head_dim, d->max_blocks_per_seq, ctas, plan.splits)
+                                              d->head_dim, d->max_blocks_per_seq, ctas)
                             .total;
     if (!workspace || workspace_bytes < need || !aligned(workspace, 256))
         return fail(SV_ERR_WORKSPACE, "workspace must be 256-byte aligned and hold %zu bytes", need);

@@ -118,11 +118,6 @@ SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
     return lo;
 }
 
-// Floats per workspace partial slot: O [rows][D], running max [rows], row sum
-// [rows], padded to 256 bytes so every slot (and every O row) is 16-byte aligned.
-__host__ __device__ inline size_t slot_stride(int rows_unit, int D) {
-    return ((size_t)rows_unit * D + 2 * (size_t)rows_unit + 63) & ~(size_t)63;
-}
 
 struct TileInfo {
     int b, hr, j, Tb;
@@ -380,10 +375,10 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 p.status[b] = (ctx_ok ? 0 : SV_FLAG_BAD_CONTEXT) | (bad ? SV_FLAG_BAD_BLOCK : 0);
         }
         // ------------------- V rows past ctx_len -------------------
-        // Softmax gives keys past ctx_len p = 0, but 0 * NaN is NaN and those
-        // rows of the last page hold whatever the pool holds; they are zeroed
-        // here once the tile has landed, off the softmax path. Every tile is
-        // released to its PV through vz, after its V has landed, so this warp
+        // Softmax gives keys past ctx_len p = 0, but 0 * NaN is NaN and the rows
+        // of the last page past ctx_len hold whatever the pool holds; they are
+        // zeroed here once the tile has landed, off the softmax path. Every tile
+        // is released to its PV through vz, after its V has landed, so this warp
         // stays within one phase of the V ring.
         TileInfo ti = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
         for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
@@ -391,10 +386,13 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const uint32_t par = (lt / NV) & 1;
             const bool landed = mbar_test(&v_full[s], par) || mbar_wait(&v_full[s], par, abort_flag, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, landed)) break;
-            const int k0 = max(0, CL[ti.b] - ti.j * TILE_KEYS);  // first key of the tile past ctx_len
-            if (k0 < TILE_KEYS) {
+            // keys [k0, k1) of the tile: past ctx_len but inside its last page (pages
+            // wholly past ctx_len were loaded as zeros by the TMA unit)
+            const int k0 = max(0, CL[ti.b] - ti.j * TILE_KEYS);
+            const int k1 = min(TILE_KEYS, (k0 + PAGE - 1) / PAGE * PAGE);
+            if (k0 < k1) {
                 uint8_t *vt = base + s * L.tile_bytes;
-                for (int e = lane; e < (TILE_KEYS - k0) * 8 * nDA; e += 32) {
+                for (int e = lane; e < (k1 - k0) * 8 * nDA; e += 32) {
                     const int key = k0 + e / (8 * nDA), rem = e - (key - k0) * (8 * nDA);
                     reinterpret_cast<uint4 *>(vt + (rem >> 3) * ATOM + key * 128)[rem & 7] = make_uint4(0, 0, 0, 0);
                 }
@@ -559,7 +557,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const int tpre = ups * TP[fb] + fhr * Tb;
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
-            const bool to_slot = nseg > 1;
+            // a cascade call leaves every unit in a slot for the shared-prefix merge
+            const bool to_slot = nseg > 1 || p.all_slots;
             float *slot = p.ws_partial + (size_t)(pend_u + blockIdx.x) * slot_floats;
             // O^T in chunks of 16 columns (few live registers)
 #pragma unroll 1
@@ -573,26 +572,11 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     for (int c = 0; c < 16; ++c) {
                         const int r = col0 + c0 + c;
                         if (r < frows) {
-                            float l = lfin[r], num = o[c];
+                            const float l = lfin[r];
+                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
                             const int ridx = frc * p.rows_unit + r;
                             const int i = ridx / p.G, hq = fh * p.G + (ridx - i * p.G);
-                            const size_t orow = ((size_t)fb * p.N + i) * p.Hq + hq;
-                            if (p.pp_o) {
-                                // cascade call: merge the row's shared-prefix partials by log-sum-exp
-                                const size_t pstride = (size_t)p.B * p.N * p.Hq;
-                                float m = mfin[r];
-                                for (int sp = 0; sp < p.pp_splits; ++sp) {
-                                    const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.pp_ml) + sp * pstride + orow);
-                                    const float op = __ldcg(p.pp_o + (sp * pstride + orow) * D + ell);
-                                    const float M = fmaxf(m, ml.x);
-                                    const float a = ex2_approx(m - M), bq = ex2_approx(ml.x - M);
-                                    num = num * a + op * bq;
-                                    l = l * a + ml.y * bq;
-                                    m = M;
-                                }
-                            }
-                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? num / l : 0.f);
-                            p.out[orow * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
+                            p.out[(((size_t)fb * p.N + i) * p.Hq + hq) * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
                         }
                     }
                 } else {
@@ -826,9 +810,6 @@ SV_DEV int block_sum_i(int v, int *red) {
 // sequence by its status warp). One CTA per (COMBINE_ROWS rows, unit), one warp
 // per row, four head dimensions per lane:
 //   M = max_k m_k,  L = sum_k 2^(m_k - M) l_k,  out = sum_k 2^(m_k - M) O_k / L.
-// In a cascade call the shared prefix's partials of the row join the merge of
-// a split unit as further terms k (a whole unit merged them in the attention
-// kernel).
 // Launched as a programmatic dependent of the attention kernel, which lets it
 // launch only after its own wait on earlier work: the schedule is recomputed
 // from ctx_lens (complete by then) before this kernel waits, so once the
@@ -854,17 +835,12 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     tot = block_sum_i(tot, red_i);
     before = block_sum_i(before, red_i);
     const int Tb = block_sum_i(own, red_i);
-    if (p.pp_o && p.status && blockIdx.x == 0 && hr == 0 && threadIdx.x == 0) {
-        griddep_wait();  // after the attention kernel's status store
-        const int f = __ldcg(p.pflag + b);
-        if (f) atomicOr(p.status + b, f);
-    }
     if (Tb == 0 || r >= rows) return;
     const int total = ups * tot;
     const int W = (total + p.num_ctas - 1) / p.num_ctas;
     const int tpre = ups * before + hr * Tb;
     const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
-    if (n == 1) return;  // written by the attention kernel (a cascade call's prefix merged there too)
+    if (n == 1) return;  // written by the attention kernel
     const int ridx = rc * RU + r;
     const int i = ridx / p.G, hq = h * p.G + (ridx - i * p.G);
     const size_t sf = slot_stride(RU, D);
@@ -886,9 +862,6 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     float M = mk;
     for (int k = lane + 32; k < n; k += 32) M = fmaxf(M, __ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r));
     M = warp_max(M);
-    const int S = p.pp_o ? p.pp_splits : 0;  // shared-prefix partials of this row
-    const size_t prow = ((size_t)b * p.N + i) * p.Hq + hq, pstride = (size_t)p.B * p.N * p.Hq;
-    for (int s = 0; s < S; ++s) M = fmaxf(M, __ldcg(p.pp_ml + 2 * (s * pstride + prow)));
     const float wl = lane < n ? exp2f(mk - M) : 0.f;  // an empty segment holds l = 0
     float L = wl * lk;
     for (int k = lane + 32; k < n; k += 32) {
@@ -897,16 +870,6 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     }
     L = warp_sum(L);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < S; ++s) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(p.pp_ml) + s * pstride + prow);
-        const float w = exp2f(ml.x - M);
-        L = fmaf(w, ml.y, L);
-        if (dl) {
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(p.pp_o + (s * pstride + prow) * D) + lane);
-            acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
-        }
-    }
 #pragma unroll
     for (int k = 0; k < COMBINE_REG_SEGS; ++k) {
         const float w = __shfl_sync(0xffffffffu, wl, k);
@@ -1080,7 +1043,7 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
         return cudaErrorInvalidValue;
     const int RP = (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess || p.all_slots) return e;  // a cascade call merges in the shared-prefix kernel
     return launch_programmatic(attn_combine_kernel, dim3((RU + COMBINE_ROWS - 1) / COMBINE_ROWS, p.units),
                                dim3(32 * COMBINE_ROWS), 0, stream, p);
 }

@@ -12,19 +12,19 @@
 //
 // Softmax over a union of key sets is the log-sum-exp merge of the softmaxes
 // over the parts, so the result is attention over the whole context:
-//   cascade_prefix_kernel  one CTA per (group, KV head, 128 group rows, prefix
-//                          split): tcgen05 products over 128-key tiles of the
-//                          shared pages, an unnormalised partial (O, running
-//                          max, row sum) per row and split; its prep warp
-//                          writes each member's suffix length and suffix block
-//                          table (its own pages after the prefix) and flags
-//                          bad block ids among the prefix pages;
+//   cascade_prep_kernel    one CTA per sequence: checks the prefix against the
+//                          context, writes the member's suffix length and
+//                          suffix block table (its own pages after the prefix)
+//                          and flags bad block ids among the group's prefix
+//                          pages;
 //   launch_attention       the split-context tcgen05 kernel over every
-//                          member's suffix (own pages, draft rows and masks);
-//                          a unit one CTA covers whole merges the rows' prefix
-//                          partials before it writes the output, a split unit
-//                          leaves slots that the combine kernel merges with
-//                          the prefix partials.
+//                          member's suffix (own pages, draft rows and masks),
+//                          every unit leaving its partial in a workspace slot;
+//   cascade_prefix_kernel  one CTA per (group, KV head, 128 group rows):
+//                          tcgen05 products over 128-key tiles of the shared
+//                          pages; its epilogue merges each row's prefix partial
+//                          (in TMEM) with the row's suffix slots and writes the
+//                          output, so no combine kernel runs.
 #include <string.h>
 
 #include "sv_internal.h"
@@ -40,24 +40,30 @@ constexpr int PF_KEYS = CASCADE_KEYS;  // keys per tile (8 pages): the N of S = 
 static_assert(PF_ROWS == 128 && PF_KEYS == 128, "the prefix pass is written for 128 x 128 tiles");
 constexpr int PF_WARP_LOAD = 0;   // TMA producer (K and V)
 constexpr int PF_WARP_MMA = 1;    // TMEM allocator and MMA issuer
-constexpr int PF_WARP_PREP = 2;   // members' suffix tables, lengths and prefix flags
-constexpr int PF_WARP_SM0 = 3;    // softmax warps 3..6: thread = row (TMEM lane quadrant = warp % 4)
-constexpr int PF_THREADS = 32 * (PF_WARP_SM0 + 4);
-constexpr int MAX_SPLITS = 8;
+constexpr int PF_WARP_SM0 = 2;    // softmax warps 2..9: quadrant warp % 4 (its TMEM lanes), half (warp - 2) / 4
+constexpr int PF_SM_WARPS = 8;
+constexpr int PF_THREADS = 32 * (PF_WARP_SM0 + PF_SM_WARPS);
+constexpr int PREP_THREADS = 128;
 constexpr uint32_t PF_ATOM = 16384;  // 128 rows x 128 bytes: one 128B-swizzle column of an operand
+constexpr uint32_t COL_S = 0;        // TMEM: S double buffer (2 x 128 columns), O (D columns),
+constexpr uint32_t COL_O = 2 * PF_KEYS;  // then exchange columns of the two warps sharing lanes
+constexpr uint32_t COL_X = COL_O + 128;
 constexpr float PF_M_NONE = -3.402823466e38f;  // running max of a row that has seen no key
 constexpr float PF_RESCALE_LOG2 = 8.f;         // O is rescaled only when a row max rises by more
 constexpr uint64_t PF_DRAIN_NS = 2000000000ull;
 
+struct PrepParams {
+    const int32_t *block_table, *ctx_lens;
+    int32_t *sfx_ctx, *sfx_table, *pflag;
+    int B, N, max_blocks, num_blocks;
+    CascadePlan plan;
+};
+
 struct PrefixParams {
     CUtensorMap tm_k, tm_v;
-    const uint16_t *q;                // bf16 bits [B][N][Hq][D]
-    const int32_t *block_table, *ctx_lens;
-    float *pp_o, *pp_ml;
-    int32_t *sfx_ctx, *sfx_table, *pflag;
-    int B, N, Hq, Hkv, G, max_blocks, num_blocks;
-    float scale_log2;
-    uint64_t wait_limit_ns;
+    AttnParams a;                     // the suffix call: slots, suffix lengths, shapes, status
+    const int32_t *block_table;       // the caller's table (the group's first member's prefix pages)
+    const int32_t *pflag;
     int NK, NV, NP;
     CascadePlan plan;
 };
@@ -74,7 +80,7 @@ __host__ __device__ inline PfLayout pf_layout(int D, int NK, int NV, int NP) {
     L.off_v = L.off_k + NK * L.tile;
     L.off_p = L.off_v + NV * L.tile;                    // P: 128 rows x 128 keys, two atoms
     L.off_bar = L.off_p + NP * 2 * PF_ATOM;
-    const int nbar = 2 * NK + 2 * NV + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 /*o*/ + 1 /*q*/ + 1 /*done*/;
+    const int nbar = 2 * NK + 2 * NV + 2 * 2 /*s*/ + 2 * NP /*p*/ + 2 /*o*/ + 1 /*q*/ + 1 /*done*/ + 4 /*pair*/;
     L.off_misc = L.off_bar + 8u * nbar;
     L.total = L.off_misc + 16u;
     return L;
@@ -98,19 +104,62 @@ SV_DEV uint32_t kmajor_off(int r, int c) {
            ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
 
-// One CTA per (group, KV head, 128 group rows, prefix split). Rows (member, i, j)
-// of every member of the group share the group's prefix pages, so each tile of
-// those pages is read once for 128 rows: S = Q K^T (M = 128 rows, N = 128 keys)
-// and O += P V (M = 128 rows, N = D) on tcgen05 with fp32 accumulators in TMEM,
-// K and V tiles by TMA (a page id outside the pool, or a page past the prefix,
+// Split-context tiles of sequence b in the suffix call (the attention kernel's rule).
+SV_DEV int suffix_tiles(const AttnParams &a, int b) {
+    const int C = __ldcg(a.ctx_lens + b);
+    return (C >= a.N && C <= a.max_blocks * PAGE) ? (C + TILE_KEYS - 1) / TILE_KEYS : 0;
+}
+
+__global__ void __launch_bounds__(PREP_THREADS) cascade_prep_kernel(const __grid_constant__ PrepParams p) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const int b = blockIdx.x;
+    const CascadePlan &pl = p.plan;
+    const int g = upper_index(pl.off, pl.num_groups, b);  // off[g] <= b < off[g+1]
+    const int P = pl.pre[g], first = pl.off[g];
+    const int C = p.ctx_lens[b];
+    const bool ok = C >= p.N && C <= p.max_blocks * PAGE && P <= C - p.N;
+    if (!ok) {  // the attention kernel flags SV_FLAG_BAD_CONTEXT and writes zeros
+        if (threadIdx.x == 0) {
+            p.sfx_ctx[b] = -1;
+            p.pflag[b] = 0;
+        }
+        return;
+    }
+    const int np = P / PAGE, ns = (C - P + PAGE - 1) / PAGE;  // np + ns <= max_blocks
+    const int32_t *own = p.block_table + (size_t)b * p.max_blocks + np;
+    int32_t *dst = p.sfx_table + (size_t)b * p.max_blocks;
+    for (int j = threadIdx.x; j < ns; j += PREP_THREADS) dst[j] = __ldg(own + j);
+    const int32_t *shared_pages = p.block_table + (size_t)first * p.max_blocks;
+    int bad = 0;
+    for (int j = threadIdx.x; j < np; j += PREP_THREADS) {
+        const int blk = __ldg(shared_pages + j);
+        bad |= blk < 0 || blk >= p.num_blocks;
+    }
+    bad = __syncthreads_or(bad);
+    if (threadIdx.x == 0) {
+        p.sfx_ctx[b] = C - P;
+        p.pflag[b] = bad ? SV_FLAG_BAD_BLOCK : 0;
+    }
+}
+
+// One CTA per (group, KV head, 128 group rows). Rows (member, i, j) of every
+// member of the group share the group's prefix pages, so each tile of those
+// pages is read once for 128 rows: S = Q K^T (M = 128 rows, N = 128 keys) and
+// O += P V (M = 128 rows, N = D) on tcgen05 with fp32 accumulators in TMEM, K
+// and V tiles by TMA (a page id outside the pool, or a page past the prefix,
 // becomes a coordinate past the pool: zeros), Q and P written into the
-// swizzled operand layout by the softmax threads. The result per row and split
-// is an unnormalised partial (O, running max m in the log2 domain, row sum l).
-// The prep warp meanwhile writes each member's suffix length and table and the
-// bad-prefix-page flags for the split-context pass that follows.
+// swizzled operand layout by the softmax threads. Two softmax warps share each
+// TMEM lane quadrant, one per half of the keys (and of the head dims of O);
+// they exchange row maxima and sums through TMEM columns, ordered by an
+// mbarrier per pair. The epilogue merges each row's prefix partial with the
+// row's suffix slots left by the split-context pass (log-sum-exp) and writes
+// the row's output.
 template <int D>
 __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __grid_constant__ PrefixParams p) {
     constexpr int nDA = D / 64;
+    constexpr int HD = D / 2;  // head dims of O per half
+    const AttnParams &a = p.a;
     const int NK = p.NK, NV = p.NV, NP = p.NP;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -122,38 +171,36 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
     uint64_t *p_full = s_empty + 2, *p_empty = p_full + NP;
     uint64_t *o_full = p_empty + NP;  // [2] by tile parity: that tile's P V has completed
     uint64_t *q_ready = o_full + 2, *done_bar = q_ready + 1;
+    uint64_t *pair_bar = done_bar + 1;  // [4] by lane quadrant: the two warps of a quadrant
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    // ---- work item -> (group, KV head, split, row tile) ----
+    // ---- work item -> (group, KV head, row tile) ----
     const CascadePlan &pl = p.plan;
     const int it = blockIdx.x;
     const int g = upper_index(pl.item0, pl.num_groups, it);
     const int b0 = pl.off[g];
-    const int NG = p.N * p.G;
+    const int G = a.G;
+    const int NG = a.N * G;
     const int rows_g = (pl.off[g + 1] - b0) * NG;
     const int tiles_g = (rows_g + PF_ROWS - 1) / PF_ROWS;
-    int rem = it - pl.item0[g];
-    const int rt = rem % tiles_g;
-    rem /= tiles_g;
-    const int s = rem % pl.splits, h = rem / pl.splits;
+    const int local = it - pl.item0[g];
+    const int rt = local % tiles_g, h = local / tiles_g;
     const int P = pl.pre[g];
-    const int nt_all = (P + PF_KEYS - 1) / PF_KEYS;
-    const int tps = (nt_all + pl.splits - 1) / pl.splits;
-    const int t0 = min(s * tps, nt_all), t1 = min(t0 + tps, nt_all);
-    const int ntiles = t1 - t0;
+    const int ntiles = (P + PF_KEYS - 1) / PF_KEYS;
 
     if (tid == 0) {
         for (int i = 0; i < NK; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
         for (int i = 0; i < NV; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], 4);
+            mbar_init(&s_full[i], 1); mbar_init(&s_empty[i], PF_SM_WARPS);
             mbar_init(&o_full[i], 1);
         }
-        for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], 4); mbar_init(&p_empty[i], 1); }
-        mbar_init(q_ready, 4);
+        for (int i = 0; i < NP; ++i) { mbar_init(&p_full[i], PF_SM_WARPS); mbar_init(&p_empty[i], 1); }
+        mbar_init(q_ready, PF_SM_WARPS);
         mbar_init(done_bar, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&pair_bar[i], 2);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -169,42 +216,44 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    // shared memory, TMEM and parameters only so far: with a programmatic launch
-    // this overlaps the previous kernel's tail
-    griddep_wait();
+    // Launched programmatically after the split-context kernel, which issues its
+    // trigger only after its own wait on everything before the call: q, the KV
+    // pools and the block table are complete when this kernel starts, so the
+    // prefix products run while the split-context kernel's last CTAs finish.
+    // Its outputs (the slots, the status) and the prep kernel's are read only
+    // after griddep_wait.
     griddep_launch_dependents();
 
     if (warp == PF_WARP_LOAD) {
         // ------------------------- TMA producer -------------------------
         if (lane == 0) {
-            const int32_t *bt = p.block_table + (size_t)b0 * p.max_blocks;  // the group's pages
+            const int32_t *bt = p.block_table + (size_t)b0 * a.max_blocks;  // the group's pages
             int issued_k = 0, issued_v = 0;
             for (int lt = 0; lt < ntiles; ++lt) {
-                const int tile = t0 + lt;
                 int blks[PF_KEYS / PAGE];
 #pragma unroll
                 for (int pg = 0; pg < PF_KEYS / PAGE; ++pg) {
-                    const int page = tile * (PF_KEYS / PAGE) + pg;
+                    const int page = lt * (PF_KEYS / PAGE) + pg;
                     const int blk = page * PAGE < P ? __ldg(bt + page) : -1;
-                    blks[pg] = (blk >= 0 && blk < p.num_blocks) ? blk : p.num_blocks;  // past the pool: zeros
+                    blks[pg] = (blk >= 0 && blk < a.num_blocks) ? blk : a.num_blocks;  // past the pool: zeros
                 }
                 const int sk = lt % NK;
-                if (!mbar_wait(&k_empty[sk], ((lt / NK) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
+                if (!mbar_wait(&k_empty[sk], ((lt / NK) & 1) ^ 1, abort_flag, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&k_full[sk], L.tile);
                 uint8_t *kd = base + L.off_k + sk * L.tile;
 #pragma unroll
                 for (int pg = 0; pg < PF_KEYS / PAGE; ++pg)
-                    for (int a = 0; a < nDA; ++a)
-                        tma_load_4d(kd + a * PF_ATOM + pg * 2048, &p.tm_k, &k_full[sk], a * 64, 0, h, blks[pg]);
+                    for (int q = 0; q < nDA; ++q)
+                        tma_load_4d(kd + q * PF_ATOM + pg * 2048, &p.tm_k, &k_full[sk], q * 64, 0, h, blks[pg]);
                 issued_k = lt + 1;
                 const int sv = lt % NV;
-                if (!mbar_wait(&v_empty[sv], ((lt / NV) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
+                if (!mbar_wait(&v_empty[sv], ((lt / NV) & 1) ^ 1, abort_flag, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&v_full[sv], L.tile);
                 uint8_t *vd = base + L.off_v + sv * L.tile;
 #pragma unroll
                 for (int pg = 0; pg < PF_KEYS / PAGE; ++pg)
-                    for (int a = 0; a < nDA; ++a)
-                        tma_load_4d(vd + a * PF_ATOM + pg * 2048, &p.tm_v, &v_full[sv], a * 64, 0, h, blks[pg]);
+                    for (int q = 0; q < nDA; ++q)
+                        tma_load_4d(vd + q * PF_ATOM + pg * 2048, &p.tm_v, &v_full[sv], q * 64, 0, h, blks[pg]);
                 issued_v = lt + 1;
             }
             if (*abort_flag) {
@@ -221,7 +270,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             constexpr uint32_t ids = idesc_bf16(128, PF_KEYS, false, false);  // Q, K both K-major
             constexpr uint32_t idp = idesc_bf16(128, D, false, true);         // P K-major, V dims-major
             const uint32_t qa = smem_u32(base + L.off_q);
-            bool ok = mbar_wait(q_ready, 0, abort_flag, p.wait_limit_ns);
+            bool ok = mbar_wait(q_ready, 0, abort_flag, a.wait_limit_ns);
             int nq = 0, np = 0;
             uint32_t idle = 0;
             uint64_t idle_since = 0;
@@ -236,7 +285,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                         for (int kk = 0; kk < D / 16; ++kk) {
                             const uint64_t ad = sw128_desc(qa + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
                             const uint64_t bd = sw128_desc(ka + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
-                            mma_bf16_ss(tmem + sb * PF_KEYS, ad, bd, ids, kk > 0);
+                            mma_bf16_ss(tmem + COL_S + sb * PF_KEYS, ad, bd, ids, kk > 0);
                         }
                         mma_commit(&s_full[sb]);
                         mma_commit(&k_empty[sk]);
@@ -254,7 +303,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                         for (int kk = 0; kk < PF_KEYS / 16; ++kk) {
                             const uint64_t ad = sw128_desc(pa + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
                             const uint64_t bd = sw128_desc(va + kk * 2048, PF_ATOM, 1024);
-                            mma_bf16_ss(tmem + 2 * PF_KEYS, ad, bd, idp, (np > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16_ss(tmem + COL_O, ad, bd, idp, (np > 0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(&o_full[np & 1]);
                         mma_commit(&p_empty[pb]);
@@ -269,90 +318,84 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     if (*abort_flag) break;
                     const uint64_t now = globaltimer_ns();
                     if (idle == 64) idle_since = now;
-                    else if (now - idle_since > p.wait_limit_ns) { *abort_flag = 1; break; }
+                    else if (now - idle_since > a.wait_limit_ns) { *abort_flag = 1; break; }
                 }
             }
             mma_commit(done_bar);  // every MMA of this CTA has finished before TMEM is freed
             mbar_wait_time(done_bar, 0, PF_DRAIN_NS);
         }
-    } else if (warp == PF_WARP_PREP) {
-        // -------- members' suffix lengths and tables, prefix page flags --------
-        // sequence b is handled by CTA b mod gridDim.x; a member whose context
-        // is invalid or shorter than its group's prefix plus N gets length -1
-        // (the attention kernel flags SV_FLAG_BAD_CONTEXT and writes zeros)
-        for (int b = blockIdx.x; b < p.B; b += gridDim.x) {
-            const int gb = upper_index(pl.off, pl.num_groups, b);
-            const int Pb = pl.pre[gb], first = pl.off[gb];
-            const int C = __ldg(p.ctx_lens + b);
-            const bool okc = C >= p.N && C <= p.max_blocks * PAGE && Pb <= C - p.N;
-            if (!okc) {
-                if (lane == 0) p.sfx_ctx[b] = -1;
-                continue;
-            }
-            const int npg = Pb / PAGE, ns = (C - Pb + PAGE - 1) / PAGE;
-            const int32_t *own = p.block_table + (size_t)b * p.max_blocks + npg;
-            int32_t *dst = p.sfx_table + (size_t)b * p.max_blocks;
-            for (int j = lane; j < ns; j += 32) dst[j] = __ldg(own + j);
-            const int32_t *shared_pages = p.block_table + (size_t)first * p.max_blocks;
-            int bad = 0;
-            for (int j = lane; j < npg; j += 32) {
-                const int blk = __ldg(shared_pages + j);
-                bad |= blk < 0 || blk >= p.num_blocks;
-            }
-            bad = __any_sync(0xffffffffu, bad);
-            if (lane == 0) {
-                p.sfx_ctx[b] = C - Pb;
-                if (bad) atomicOr(p.pflag + b, SV_FLAG_BAD_BLOCK);
-            }
-        }
     } else {
-        // ------------------- softmax: one thread per row -------------------
-        const int quad = warp & 3;              // TMEM lane quadrant of this warp
-        const int ell = quad * 32 + lane;       // row of the tile = TMEM lane
+        // --------- softmax: two warps per lane quadrant, a thread per row ---------
+        const int quad = warp & 3;                   // TMEM lane quadrant of this warp
+        const int half = (warp - PF_WARP_SM0) >> 2;  // keys [64 half, +64), O dims [HD half, +HD)
+        const int ell = quad * 32 + lane;            // row of the tile = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        const int r = rt * PF_ROWS + ell;       // group row (member, i, j)
-        long long prow = -1;                    // row (b, i, hq) of q / out
+        const int r = rt * PF_ROWS + ell;            // group row (member, i, j)
+        int mb = -1, mi = 0, mj = 0;                 // its sequence, query row and head offset
         if (r < rows_g) {
-            const int m = r / NG, rr = r - m * NG, i = rr / p.G, j = rr - i * p.G;
-            prow = ((long long)(b0 + m) * p.N + i) * p.Hq + (long long)h * p.G + j;
+            const int m = r / NG, rr = r - m * NG;
+            mb = b0 + m;
+            mi = rr / G;
+            mj = rr - mi * G;
         }
+        const long long prow = mb < 0 ? -1 : ((long long)mb * a.N + mi) * a.Hq + (long long)h * G + mj;
         auto warp_arrive = [&](uint64_t *b) {
             __syncwarp();
             if (lane == 0) mbar_arrive(b);
         };
         auto wait_w = [&](uint64_t *b, uint32_t parity) -> bool {
-            const bool ok = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, p.wait_limit_ns);
-            return __all_sync(0xffffffffu, ok);
+            const bool okw = mbar_test(b, parity) || mbar_wait(b, parity, abort_flag, a.wait_limit_ns);
+            return __all_sync(0xffffffffu, okw);
         };
-        {   // Q row into the swizzled K-major operand tile (zeros past the group's rows)
-            const uint4 *src = reinterpret_cast<const uint4 *>(p.q + (prow < 0 ? 0 : prow) * D);
+        // the two warps of a quadrant swap one value per row through TMEM
+        // columns COL_X + 2 slot + half (the partner writes the other one)
+        uint32_t pair_phase = 0;
+        auto swap = [&](float v, int slot, bool &okx) -> float {
+            tmem_st1(lane_base + COL_X + 2 * slot + half, v);
+            tmem_wait_st();
+            tc_fence_before();
+            warp_arrive(&pair_bar[quad]);
+            okx = okx && wait_w(&pair_bar[quad], pair_phase);
+            pair_phase ^= 1;
+            tc_fence_after();
+            return tmem_ld1(lane_base + COL_X + 2 * slot + (half ^ 1));
+        };
+        {   // Q row (this half's head dims) into the swizzled K-major operand tile
+            const uint4 *src = reinterpret_cast<const uint4 *>(a.q + (prow < 0 ? 0 : prow) * D);
             uint8_t *qt = base + L.off_q;
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c) {
+            for (int c = half * (D / 16); c < (half + 1) * (D / 16); ++c) {
                 const uint4 v = prow >= 0 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
                 *reinterpret_cast<uint4 *>(qt + kmajor_off(ell, c)) = v;
             }
             fence_proxy_async_smem();
             warp_arrive(q_ready);
         }
-        const float sc = p.scale_log2;
-        float m_run = PF_M_NONE, l_run = 0.f;
+        const float sc = a.scale_log2;
+        float m_run = PF_M_NONE, l_run = 0.f;  // l_run: this half's keys only
         bool ok = true;
         for (int lt = 0; lt < ntiles && ok; ++lt) {
             const int sb = lt & 1, pb = lt % NP;
-            const int valid = P - (t0 + lt) * PF_KEYS;  // keys of this tile inside the prefix
+            const int valid = P - lt * PF_KEYS - half * 64;  // keys of this half inside the prefix
             if (!(ok = wait_w(&s_full[sb], (lt >> 1) & 1))) break;
             tc_fence_after();
-            const uint32_t sa = lane_base + sb * PF_KEYS;
+            const uint32_t sa = lane_base + COL_S + sb * PF_KEYS + half * 64;
             float mx = -INFINITY;
-#pragma unroll 1
-            for (int c0 = 0; c0 < PF_KEYS; c0 += 32) {
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 32) {
                 float v[32];
                 tmem_ld32(sa + c0, v);
                 tmem_wait_ld();
+                if (valid >= 64) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) mx = fmaxf(mx, c0 + c < valid ? v[c] : -INFINITY);
+                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, v[c]);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, c0 + c < valid ? v[c] : -INFINITY);
+                }
             }
+            mx = fmaxf(mx, swap(mx, lt & 1, ok));
+            if (!ok) break;
             // the running max is raised on a row's first tile, or when a score
             // beats it by more than 2^8; otherwise the tile folds in as it is
             const float cand = mx * sc;
@@ -361,40 +404,44 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             const float alpha = ex2_approx(m_run - m_new);  // first tile: 0; unchanged: 1
             l_run *= alpha;
             if (lt > 0 && __any_sync(0xffffffffu, raise)) {
-                // O (this row, every dim) scaled once the previous tile's P V has landed
+                // this half's dims of O, once the previous tile's P V has landed
                 if (!(ok = wait_w(&o_full[(lt - 1) & 1], ((lt - 1) >> 1) & 1))) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 16) {
+#pragma unroll
+                for (int c0 = 0; c0 < HD; c0 += 16) {
                     float o[16];
-                    tmem_ld16(lane_base + 2 * PF_KEYS + c0, o);
+                    tmem_ld16(lane_base + COL_O + half * HD + c0, o);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c = 0; c < 16; ++c) o[c] *= alpha;
-                    tmem_st16(lane_base + 2 * PF_KEYS + c0, o);
+                    tmem_st16(lane_base + COL_O + half * HD + c0, o);
                 }
                 tmem_wait_st();
             }
             m_run = m_new;
             if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
             uint8_t *pt = base + L.off_p + pb * 2 * PF_ATOM;
-#pragma unroll 1
-            for (int c0 = 0; c0 < PF_KEYS; c0 += 32) {
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 32) {
                 float v[32];
                 tmem_ld32(sa + c0, v);
                 tmem_wait_ld();
                 uint32_t pk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const float p0 = c0 + c < valid ? ex2_approx(fmaf(v[c], sc, -m_run)) : 0.f;
-                    const float p1 = c0 + c + 1 < valid ? ex2_approx(fmaf(v[c + 1], sc, -m_run)) : 0.f;
+                    float p0 = ex2_approx(fmaf(v[c], sc, -m_run));
+                    float p1 = ex2_approx(fmaf(v[c + 1], sc, -m_run));
+                    if (valid < 64) {
+                        p0 = c0 + c < valid ? p0 : 0.f;
+                        p1 = c0 + c + 1 < valid ? p1 : 0.f;
+                    }
                     l_run += p0 + p1;
                     const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
                     pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&hv);
                 }
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(pt + kmajor_off(ell, (c0 >> 3) + q4)) =
+                    *reinterpret_cast<uint4 *>(pt + kmajor_off(ell, half * 8 + (c0 >> 3) + q4)) =
                         make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
             }
             tc_fence_before();
@@ -402,36 +449,115 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             fence_proxy_async_smem();
             warp_arrive(&p_full[pb]);
         }
-        // ---- partial of this row and split: O unnormalised, (m, l) ----
-        const size_t pstride = (size_t)p.B * p.N * p.Hq;
-        float *dst = prow >= 0 ? p.pp_o + ((size_t)s * pstride + (size_t)prow) * D : nullptr;
+        // ---- epilogue: prefix partial (O in TMEM, m_run, l) merged with the row's suffix slots ----
+        griddep_wait();  // the split-context kernel has completed: its slots are visible
         if (ok && ntiles > 0) ok = wait_w(&o_full[(ntiles - 1) & 1], ((ntiles - 1) >> 1) & 1);
-        if (ok && ntiles > 0) {
+        if (ok) {
             tc_fence_after();
-#pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 16) {
-                float o[16];
-                tmem_ld16(lane_base + 2 * PF_KEYS + c0, o);
-                tmem_wait_ld();
-                if (dst)
+            const float lo = swap(l_run, 2, ok);
+            const float l_p = half == 0 ? l_run + lo : lo + l_run;  // the same sum in both halves
+            const float m_p = ntiles > 0 ? m_run : PF_M_NONE;
+            // split-context schedule of the suffix call (the attention kernel's
+            // rule): the sequences' tile prefix, one copy per warp, in the P
+            // buffers, which the last P V has finished reading
+            int *TP = reinterpret_cast<int *>(base + L.off_p) + (warp - PF_WARP_SM0) * (MAX_SEQS + 1);
+            {
+                const int per = (a.B + 31) / 32;
+                const int s0 = min(lane * per, a.B), s1 = min(s0 + per, a.B);
+                int loc = 0;
+                for (int b = s0; b < s1; ++b) loc += suffix_tiles(a, b);
+                int incl = loc;
 #pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4)
-                        *reinterpret_cast<float4 *>(dst + c0 + 4 * c4) =
-                            make_float4(o[4 * c4], o[4 * c4 + 1], o[4 * c4 + 2], o[4 * c4 + 3]);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                int run = incl - loc;
+                for (int b = s0; b < s1; ++b) {
+                    TP[b] = run;
+                    run += suffix_tiles(a, b);
+                }
+                if (lane == 31) TP[a.B] = incl;
+                __syncwarp();
             }
-        } else if (dst) {
-            for (int c = 0; c < D; c += 4) *reinterpret_cast<float4 *>(dst + c) = make_float4(0.f, 0.f, 0.f, 0.f);
-            m_run = PF_M_NONE;
-            l_run = 0.f;
+            const int ups = a.Hkv * a.RC;
+            const int total = ups * TP[a.B];
+            const int W = total > 0 ? (total + a.num_ctas - 1) / a.num_ctas : 1;
+            const size_t sf = slot_stride(a.rows_unit, D);
+            int n = 0, ru = 0;
+            const float *seg = a.ws_partial;
+            if (mb >= 0) {
+                const int Nc = a.rows_unit / G;  // whole query rows per row chunk
+                const int rc = mi / Nc;          // row chunk of the unit that holds query row mi
+                ru = (mi - rc * Nc) * G + mj;
+                const int Tb = TP[mb + 1] - TP[mb];
+                if (Tb > 0) {
+                    const int hr = h * a.RC + rc;
+                    const int u = mb * ups + hr;
+                    const int tpre = ups * TP[mb] + hr * Tb;
+                    const int first = tpre / W;
+                    n = (tpre + Tb - 1) / W - first + 1;
+                    seg = a.ws_partial + (size_t)(u + first) * sf;
+                }
+            }
+            // weights of the prefix partial and of the n suffix segments
+            const size_t ml_off = (size_t)a.rows_unit * D + ru;
+            float M = m_p;
+            for (int k = 0; k < n; ++k) M = fmaxf(M, __ldcg(seg + k * sf + ml_off));
+            const float wp = ex2_approx(m_p - M);  // M_NONE - finite underflows to 0
+            float Lsum = wp * l_p;
+            for (int k = 0; k < n; ++k)
+                Lsum += ex2_approx(__ldcg(seg + k * sf + ml_off) - M) * __ldcg(seg + k * sf + ml_off + a.rows_unit);
+            const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll 1
+            for (int c0 = 0; c0 < HD; c0 += 16) {
+                float o[16];
+                tmem_ld16(lane_base + COL_O + half * HD + c0, o);
+                tmem_wait_ld();
+                if (n > 0) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) o[c] = ntiles > 0 ? o[c] * wp : 0.f;
+                    for (int k = 0; k < n; ++k) {
+                        const float wk = ex2_approx(__ldcg(seg + k * sf + ml_off) - M);
+                        const float4 *src = reinterpret_cast<const float4 *>(seg + k * sf + (size_t)ru * D + half * HD + c0);
+#pragma unroll
+                        for (int c4 = 0; c4 < 4; ++c4) {
+                            const float4 x = __ldcg(src + c4);
+                            o[4 * c4] = fmaf(wk, x.x, o[4 * c4]);
+                            o[4 * c4 + 1] = fmaf(wk, x.y, o[4 * c4 + 1]);
+                            o[4 * c4 + 2] = fmaf(wk, x.z, o[4 * c4 + 2]);
+                            o[4 * c4 + 3] = fmaf(wk, x.w, o[4 * c4 + 3]);
+                        }
+                    }
+                    uint32_t pk[8];
+#pragma unroll
+                    for (int c = 0; c < 16; c += 2) {
+                        const __nv_bfloat162 hv = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
+                        pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&hv);
+                    }
+                    uint4 *dst = reinterpret_cast<uint4 *>(a.out + (size_t)prow * D + half * HD + c0);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
         }
-        if (dst) *reinterpret_cast<float2 *>(p.pp_ml + 2 * ((size_t)s * pstride + (size_t)prow)) = make_float2(m_run, l_run);
     }
 
     // ----------------------------- teardown -------------------------------
     tc_fence_before();
     __syncthreads();
-    if (*abort_flag && tid < 32)
-        for (int b = lane; b < p.B; b += 32) atomicOr(p.pflag + b, SV_FLAG_TIMEOUT);
+    if (a.status && tid < 32) {
+        // flags of the group's members, after the split-context kernel's status
+        // stores: bad prefix pages (the first row tile of head 0 reports them),
+        // and a wait of this CTA that gave up
+        griddep_wait();
+        const bool report = rt == 0 && h == 0;
+        const int aborted = *abort_flag;
+        for (int b = b0 + lane; b < pl.off[g + 1]; b += 32) {
+            const int f = (report ? __ldcg(p.pflag + b) : 0) | (aborted ? SV_FLAG_TIMEOUT : 0);
+            if (f) atomicOr(a.status + b, f);
+        }
+    }
     if (warp == PF_WARP_MMA) {
         __syncwarp();
         tc_fence_after();
@@ -445,35 +571,23 @@ constexpr int PF_SMEM_LIMIT = 227 * 1024;
 
 }  // namespace
 
-void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, int num_sms, CascadePlan *pl) {
+void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, CascadePlan *pl) {
     memset(pl, 0, sizeof *pl);
     const int G = Hq / Hkv;
     pl->num_groups = cd->num_groups;
-    int base = 0, max_tiles = 0;
     for (int g = 0; g <= cd->num_groups; ++g) pl->off[g] = cd->group_offsets[g];
-    for (int g = 0; g < cd->num_groups; ++g) {
-        pl->pre[g] = cd->prefix_lens[g];
-        const int rows = (pl->off[g + 1] - pl->off[g]) * N * G;
-        base += (rows + CASCADE_ROWS - 1) / CASCADE_ROWS * Hkv;
-        max_tiles = max(max_tiles, (pl->pre[g] + CASCADE_KEYS - 1) / CASCADE_KEYS);
-    }
-    // One CTA per SM (shared memory and TMEM): the most prefix splits whose
-    // items still fit one wave. Every split adds a partial per row.
-    int S = base > 0 ? num_sms / base : 1;
-    S = max(1, min(S, min(MAX_SPLITS, max(1, max_tiles))));
-    pl->splits = S;
     int acc = 0;
     for (int g = 0; g < cd->num_groups; ++g) {
+        pl->pre[g] = cd->prefix_lens[g];
         pl->item0[g] = acc;
         const int rows = (pl->off[g + 1] - pl->off[g]) * N * G;
-        acc += (rows + CASCADE_ROWS - 1) / CASCADE_ROWS * Hkv * S;
+        acc += (rows + CASCADE_ROWS - 1) / CASCADE_ROWS * Hkv;
     }
     pl->item0[cd->num_groups] = acc;
     pl->items = acc;
 }
 
-CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max_blocks, int num_ctas,
-                                   int splits) {
+CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max_blocks, int num_ctas) {
     CascadeWorkspace w;
     size_t off = 0;
     w.slots = off;
@@ -484,13 +598,24 @@ CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max
     off += align256((size_t)B * sizeof(int32_t));
     w.sfx_table = off;
     off += align256((size_t)B * max_blocks * sizeof(int32_t));
-    const size_t rows = (size_t)splits * B * N * Hq;
-    w.pp_o = off;
-    off += align256(rows * D * sizeof(float));
-    w.pp_ml = off;
-    off += align256(rows * 2 * sizeof(float));
     w.total = off;
     return w;
+}
+
+template <typename Params>
+static cudaError_t launch_pdl(void (*kfn)(Params), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              const Params &prm) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kfn, prm);
 }
 
 template <int D>
@@ -506,71 +631,57 @@ static cudaError_t launch_prefix(PrefixParams &fp, int items, cudaStream_t strea
     fp.NK = choices[k][0];
     fp.NV = choices[k][1];
     fp.NP = choices[k][2];
+    // the epilogue keeps one copy of the sequences' tile prefix per softmax warp in the P buffers
+    if ((size_t)PF_SM_WARPS * (MAX_SEQS + 1) * sizeof(int) > (size_t)fp.NP * 2 * PF_ATOM)
+        return cudaErrorInvalidConfiguration;
     const size_t smem = L.total + 1024;
     auto kfn = cascade_prefix_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)items);
-    cfg.blockDim = dim3(PF_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kfn, fp);
+    return launch_pdl(kfn, dim3((unsigned)items), dim3(PF_THREADS), smem, stream, fp);
 }
 
 cudaError_t launch_cascade(const AttnParams &p, const CascadePlan &plan, cudaStream_t stream) {
-    const CascadeWorkspace w = cascade_workspace(p.B, p.N, p.Hq, p.Hkv, p.D, p.max_blocks, p.num_ctas, plan.splits);
+    const CascadeWorkspace w = cascade_workspace(p.B, p.N, p.Hq, p.Hkv, p.D, p.max_blocks, p.num_ctas);
     char *base = reinterpret_cast<char *>(p.ws_partial);
     int32_t *sfx_ctx = reinterpret_cast<int32_t *>(base + w.sfx_ctx);
     int32_t *pflag = reinterpret_cast<int32_t *>(base + w.pflag);
     int32_t *sfx_table = reinterpret_cast<int32_t *>(base + w.sfx_table);
-    float *pp_o = reinterpret_cast<float *>(base + w.pp_o);
-    float *pp_ml = reinterpret_cast<float *>(base + w.pp_ml);
 
-    // prefix flags are ORed in by the prefix kernel's CTAs
-    cudaError_t e = cudaMemsetAsync(pflag, 0, (size_t)p.B * sizeof(int32_t), stream);
+    PrepParams pp;
+    pp.block_table = p.block_table;
+    pp.ctx_lens = p.ctx_lens;
+    pp.sfx_ctx = sfx_ctx;
+    pp.sfx_table = sfx_table;
+    pp.pflag = pflag;
+    pp.B = p.B;
+    pp.N = p.N;
+    pp.max_blocks = p.max_blocks;
+    pp.num_blocks = p.num_blocks;
+    pp.plan = plan;
+    cudaError_t e = launch_pdl(cascade_prep_kernel, dim3((unsigned)p.B), dim3(PREP_THREADS), 0, stream, pp);
     if (e != cudaSuccess) return e;
 
+    // the members' suffixes: every unit leaves its partial in a slot
+    AttnParams a = p;
+    a.block_table = sfx_table;
+    a.ctx_lens = sfx_ctx;
+    a.ws_partial = reinterpret_cast<float *>(base + w.slots);
+    a.all_slots = 1;
+    e = launch_attention(a, stream);
+    if (e != cudaSuccess) return e;
+
+    // the shared prefixes, merged with the slots into the output
     PrefixParams fp;
     memset(&fp, 0, sizeof fp);
     if (!encode_pool_map(&fp.tm_k, p.k_pool, p.num_blocks, p.Hkv, p.D) ||
         !encode_pool_map(&fp.tm_v, p.v_pool, p.num_blocks, p.Hkv, p.D))
         return cudaErrorInvalidValue;
-    fp.q = p.q;
+    fp.a = a;
     fp.block_table = p.block_table;
-    fp.ctx_lens = p.ctx_lens;
-    fp.pp_o = pp_o;
-    fp.pp_ml = pp_ml;
-    fp.sfx_ctx = sfx_ctx;
-    fp.sfx_table = sfx_table;
     fp.pflag = pflag;
-    fp.B = p.B;
-    fp.N = p.N;
-    fp.Hq = p.Hq;
-    fp.Hkv = p.Hkv;
-    fp.G = p.G;
-    fp.max_blocks = p.max_blocks;
-    fp.num_blocks = p.num_blocks;
-    fp.scale_log2 = p.scale_log2;
-    fp.wait_limit_ns = p.wait_limit_ns;
     fp.plan = plan;
-    e = p.D == 128 ? launch_prefix<128>(fp, plan.items, stream) : launch_prefix<64>(fp, plan.items, stream);
-    if (e != cudaSuccess) return e;
-
-    AttnParams a = p;
-    a.block_table = sfx_table;
-    a.ctx_lens = sfx_ctx;
-    a.ws_partial = reinterpret_cast<float *>(base + w.slots);
-    a.pp_o = pp_o;
-    a.pp_ml = pp_ml;
-    a.pflag = pflag;
-    a.pp_splits = plan.splits;
-    return launch_attention(a, stream);
+    return p.D == 128 ? launch_prefix<128>(fp, plan.items, stream) : launch_prefix<64>(fp, plan.items, stream);
 }
 
 }  // namespace sv

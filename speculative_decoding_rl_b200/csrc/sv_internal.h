@@ -27,6 +27,7 @@ struct AcceptParams {
     int B, N, V, S;        // S = slices per row
     float log2e_over_T;    // log2(e) / T for T > 0
     int greedy;
+    int vec;               // V % 4 == 0 and 16-byte aligned rows: 16-byte loads
     struct { uint32_t k0, k1; } key;
     int8_t parent[64];
     void *workspace;       // accept_workspace_bytes(B, N, V), 256-byte aligned
@@ -63,13 +64,9 @@ struct AttnParams {
     int units;                 // B * Hkv * RC
     int num_ctas;
     float scale_log2;          // log2(e) / sqrt(D)
-    // Cascade call (null pp_o: a plain call). Every unit then leaves a slot,
-    // and the combine kernel folds in pp_splits partials of the shared prefix
-    // per row and ORs pflag into the status.
-    const float *pp_o;         // [pp_splits][B][N][Hq][D] unnormalised O
-    const float *pp_ml;        // [pp_splits][B][N][Hq][2] running max (log2 domain), row sum
-    const int32_t *pflag;      // [B] status bits found on the prefix pages
-    int pp_splits;
+    // Cascade call: every unit leaves its partial in a slot and no combine
+    // kernel runs; the shared-prefix kernel that follows merges each row.
+    int all_slots;
     // Bound of every device-side wait (2 s). Test hooks shorten it, and with
     // stall set make one wait per CTA run out (see sv_testing_*).
     uint64_t wait_limit_ns;
@@ -77,6 +74,14 @@ struct AttnParams {
 };
 
 size_t attention_workspace_bytes(int B, int N, int Hq, int Hkv, int D, int num_ctas);
+#ifdef __CUDACC__
+// Floats per workspace partial slot: O [rows][D], running max [rows], row sum
+// [rows], padded to 256 bytes so every slot (and every O row) is 16-byte aligned.
+// The partial of a unit's k-th CTA segment is slot unit + (first CTA) + k.
+__host__ __device__ inline size_t slot_stride(int rows_unit, int D) {
+    return ((size_t)rows_unit * D + 2 * (size_t)rows_unit + 63) & ~(size_t)63;
+}
+#endif
 // TMA map of a K or V pool [num_blocks][Hkv][16][D]: boxes of 16 keys x 64 dims,
 // 128-byte swizzled (whole_page: 16 keys x D, unswizzled). A block id of
 // num_blocks addresses past the pool and loads zeros.
@@ -88,26 +93,25 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream);
 
 // ------------------------------ cascade ------------------------------------
 // Shared-prefix pass: one CTA of CASCADE_ROWS query rows per (group, KV head,
-// row tile, prefix split), CASCADE_KEYS keys per tile.
+// row tile), CASCADE_KEYS keys per tile.
 constexpr int CASCADE_ROWS = 128;
 constexpr int CASCADE_KEYS = 128;
 
 struct CascadePlan {
-    int num_groups, splits, items;
+    int num_groups, items;
     int off[SV_CASCADE_MAX_GROUPS + 1];    // group member offsets
     int pre[SV_CASCADE_MAX_GROUPS];        // shared keys per group
     int item0[SV_CASCADE_MAX_GROUPS + 1];  // first work item of each group
 };
 
-// Work items and prefix splits for a validated cascade descriptor.
-void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, int num_sms, CascadePlan *plan);
-// Workspace: the attention slots, then suffix lengths, prefix flags, suffix
-// block table and the prefix partials, each 256-byte aligned.
+// Work items of a validated cascade descriptor.
+void cascade_plan(const sv_cascade_desc *cd, int N, int Hq, int Hkv, CascadePlan *plan);
+// Workspace: the attention slots, then suffix lengths, prefix flags and the
+// suffix block table, each 256-byte aligned.
 struct CascadeWorkspace {
-    size_t slots, sfx_ctx, pflag, sfx_table, pp_o, pp_ml, total;
+    size_t slots, sfx_ctx, pflag, sfx_table, total;
 };
-CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max_blocks, int num_ctas,
-                                   int splits);
+CascadeWorkspace cascade_workspace(int B, int N, int Hq, int Hkv, int D, int max_blocks, int num_ctas);
 // p describes the whole call with the caller's block table and lengths; p's
 // workspace pointer is the base of a CascadeWorkspace.
 cudaError_t launch_cascade(const AttnParams &p, const CascadePlan &plan, cudaStream_t stream);

@@ -234,6 +234,16 @@ SV_DEV void tmem_st16(uint32_t taddr, const float *v) {
 }
 SV_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// One column: 32 lanes x 32 bits (one value per thread of the warp).
+SV_DEV float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
+SV_DEV void tmem_st1(uint32_t taddr, float v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
+
 // Load NC consecutive columns (NC a multiple of 8) into v.
 template <int NC>
 SV_DEV void tmem_ld_cols(uint32_t taddr, float *v) {
