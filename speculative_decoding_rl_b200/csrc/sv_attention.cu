@@ -77,15 +77,25 @@ SV_DEV int seq_tiles(const AttnParams &p, int b) {
     return ok ? (C + TILE_KEYS - 1) / TILE_KEYS : 0;
 }
 
-// Exclusive prefix of per-sequence tile counts into TP[0..B] (and, when CL is
-// given, the context lengths into CL[0..B)); the whole block participates.
+// Schedule positions of one unit of sequence b: its tiles plus UNIT_COST.
+SV_DEV int seq_slots(const AttnParams &p, int b) {
+    const int t = seq_tiles(p, b);
+    return t > 0 ? t + UNIT_COST : 0;
+}
+
+// Tiles of a sequence from its schedule positions.
+SV_DEV int real_tiles(int positions) { return positions > 0 ? positions - UNIT_COST : 0; }
+
+// Exclusive prefix of per-sequence schedule positions (seq_slots) into
+// TP[0..B] (and, when CL is given, the context lengths into CL[0..B)); the
+// whole block participates.
 SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch, int *CL = nullptr) {
     const int nt = blockDim.x, tid = threadIdx.x;
     const int per = (p.B + nt - 1) / nt;
     const int s0 = min(tid * per, p.B), s1 = min(s0 + per, p.B);
     int local = 0;
     for (int b = s0; b < s1; ++b) {
-        local += seq_tiles(p, b);
+        local += seq_slots(p, b);
         if (CL) CL[b] = p.ctx_lens[b];
     }
     const int lane = tid & 31, warp = tid >> 5;
@@ -102,13 +112,13 @@ SV_DEV void tile_prefix(const AttnParams &p, int *TP, int *scratch, int *CL = nu
     int run = wpre + incl - local;
     for (int b = s0; b < s1; ++b) {
         TP[b] = run;
-        run += seq_tiles(p, b);
+        run += seq_slots(p, b);
     }
     if (tid == nt - 1) TP[p.B] = run;
     __syncthreads();
 }
 
-// Tile t -> sequence b (largest b with ups*TP[b] <= t).
+// Schedule position t -> sequence b (largest b with ups*TP[b] <= t).
 SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
     int lo = 0, hi = B;
     while (hi - lo > 1) {
@@ -118,20 +128,10 @@ SV_DEV int tile_seq(const int *TP, int B, int ups, int t) {
     return lo;
 }
 
-
+// A tile: sequence b, head/row-chunk hr, tile j of the unit's Tb tiles.
 struct TileInfo {
     int b, hr, j, Tb;
 };
-
-SV_DEV TileInfo decode_tile(const int *TP, int B, int ups, int t) {
-    TileInfo ti;
-    ti.b = tile_seq(TP, B, ups, t);
-    ti.Tb = TP[ti.b + 1] - TP[ti.b];
-    const int off = t - ups * TP[ti.b];
-    ti.hr = off / ti.Tb;
-    ti.j = off - ti.hr * ti.Tb;
-    return ti;
-}
 
 // The tile after ti in the end-to-end order (j, then head/row chunk, then
 // sequence; sequences without tiles are skipped). Callers stop at their range's
@@ -143,8 +143,38 @@ SV_DEV void next_tile(TileInfo &ti, const int *TP, int B, int ups) {
     ti.hr = 0;
     do {
         ++ti.b;
-        ti.Tb = ti.b < B ? TP[ti.b + 1] - TP[ti.b] : 1;
+        ti.Tb = ti.b < B ? real_tiles(TP[ti.b + 1] - TP[ti.b]) : 1;
     } while (ti.b < B && ti.Tb == 0);
+}
+
+// The first tile a CTA owns and how many it owns: the tiles whose schedule
+// positions fall in [v0, v1) (positions past a unit's tiles hold no work).
+SV_DEV TileInfo cta_tiles(const int *TP, int B, int ups, int v0, int v1, int *ntiles) {
+    TileInfo ti{0, 0, 0, 1};
+    *ntiles = 0;
+    if (v0 >= v1) return ti;
+    ti.b = tile_seq(TP, B, ups, v0);
+    const int T1 = TP[ti.b + 1] - TP[ti.b];  // positions per unit of b (> 0)
+    const int off = v0 - ups * TP[ti.b];
+    ti.hr = off / T1;
+    ti.j = off - ti.hr * T1;
+    ti.Tb = real_tiles(T1);
+    if (ti.j >= ti.Tb) {  // a position past the unit's tiles: start at the next unit
+        ti.j = ti.Tb - 1;
+        next_tile(ti, TP, B, ups);
+    }
+    TileInfo w = ti;
+    int n = 0;
+    while (w.b < B) {
+        const int pos = ups * TP[w.b] + w.hr * (w.Tb + UNIT_COST) + w.j;
+        if (pos >= v1) break;
+        const int here = min(w.Tb - w.j, v1 - pos);
+        n += here;
+        w.j = w.Tb - 1;
+        next_tile(w, TP, B, ups);
+    }
+    *ntiles = n;
+    return ti;
 }
 
 // ---------------------------------------------------------------------------
@@ -284,18 +314,24 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     griddep_wait();
     griddep_launch_dependents();  // the combine kernel may now be scheduled
     tile_prefix(p, TP, scratch, CL);  // contains __syncthreads
+    const int ups = p.Hkv * p.RC;
+    const int total = ups * TP[p.B];  // schedule positions of all units
+    const int W = total > 0 ? (total + p.num_ctas - 1) / p.num_ctas : 1;
+    if (tid == 0) {
+        // this CTA's tiles: those at positions [cta*W, cta*W + W); published to
+        // every role through the (now free) scratch words
+        const int v0 = min((int)blockIdx.x * W, total), v1 = min(v0 + W, total);
+        int n;
+        const TileInfo t0 = cta_tiles(TP, p.B, ups, v0, v1, &n);
+        scratch[0] = t0.b; scratch[1] = t0.hr; scratch[2] = t0.j; scratch[3] = t0.Tb; scratch[4] = n;
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    const int ups = p.Hkv * p.RC;
-    const int total = ups * TP[p.B];
-    const int W = total > 0 ? (total + p.num_ctas - 1) / p.num_ctas : 1;
-    const int t_begin = min((int)blockIdx.x * W, total);
-    const int t_end = min(t_begin + W, total);
-    const int ntiles = t_end - t_begin;
+    const TileInfo t_first{scratch[0], scratch[1], scratch[2], scratch[3]};
+    const int ntiles = scratch[4];
 
     if (warp == WARP_K || warp == WARP_V) {
         // ------------------- TMA producers (Q and K; V) -------------------
@@ -308,7 +344,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             uint8_t *ring = base + (is_k ? L.off_k : 0u);
             const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
             int lu = -1, issued_tiles = 0;
-            TileInfo ti = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+            TileInfo ti = t_first;
             for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
                 const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
                 // gather the tile's page ids first (independent loads), then wait for the slot
@@ -380,7 +416,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         // zeroed here once the tile has landed, off the softmax path. Every tile
         // is released to its PV through vz, after its V has landed, so this warp
         // stays within one phase of the V ring.
-        TileInfo ti = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+        TileInfo ti = t_first;
         for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
             const int s = lt % NV;
             const uint32_t par = (lt / NV) & 1;
@@ -412,7 +448,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             constexpr uint32_t idq = idesc_bf16(128, RP, false, false);
             constexpr uint32_t idp = idesc_bf16(128, RP, true, true);
             int nq = 0, np = 0, lu = -1, qb = 0, lup = -1;
-            TileInfo tq = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+            TileInfo tq = t_first;
             TileInfo tp = tq;
             uint32_t idle = 0;
             uint64_t idle_since = 0;
@@ -553,8 +589,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const int fb = pend_u / ups, fhr = pend_u - fb * ups;
             const int fh = fhr / p.RC, frc = fhr - fh * p.RC;
             const int frows = min(p.rows_unit, p.R - frc * p.rows_unit);
-            const int Tb = TP[fb + 1] - TP[fb];
-            const int tpre = ups * TP[fb] + fhr * Tb;
+            const int Tb = real_tiles(TP[fb + 1] - TP[fb]);
+            const int tpre = ups * TP[fb] + fhr * (Tb + UNIT_COST);  // the unit's first position
             const int first_cta = tpre / W;
             const int nseg = (tpre + Tb - 1) / W - first_cta + 1;
             // a cascade call leaves every unit in a slot for the shared-prefix merge
@@ -568,15 +604,19 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 tmem_wait_ld();
                 if (ell >= D) continue;
                 if (!to_slot) {
+                    // row r of the unit is query row frc*Nc + r/G, head fh*G + r%G;
+                    // rowi holds r/G (no division here: this code runs once per
+                    // unit and is kept short)
+                    uint16_t *orow = p.out + (((size_t)fb * p.N + frc * P.Nc) * p.Hq + fh * p.G) * D + ell;
+                    const size_t hqd = (size_t)p.Hq * D;
 #pragma unroll
                     for (int c = 0; c < 16; ++c) {
                         const int r = col0 + c0 + c;
                         if (r < frows) {
+                            const int i = rowi[r];
                             const float l = lfin[r];
-                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? o[c] / l : 0.f);
-                            const int ridx = frc * p.rows_unit + r;
-                            const int i = ridx / p.G, hq = fh * p.G + (ridx - i * p.G);
-                            p.out[(((size_t)fb * p.N + i) * p.Hq + hq) * D + ell] = *reinterpret_cast<const uint16_t *>(&v);
+                            const __nv_bfloat16 v = __float2bfloat16_rn(l > 0.f ? __fdividef(o[c], l) : 0.f);
+                            orow[i * hqd + (size_t)(r - i * p.G) * D] = *reinterpret_cast<const uint16_t *>(&v);
                         }
                     }
                 } else {
@@ -600,7 +640,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         if (p.stall) ok = wait_w(stall_bar, 0);
 
         // one pass past the last tile closes and finishes the CTA's last unit
-        TileInfo tnext = ntiles > 0 ? decode_tile(TP, p.B, ups, t_begin) : TileInfo{0, 0, 0, 1};
+        TileInfo tnext = t_first;
         for (int lt = 0; lt <= ntiles && ok; ++lt) {
             const bool end = lt == ntiles;
             const TileInfo ti = end ? TileInfo{0, 0, 0, 1} : tnext;
@@ -824,13 +864,14 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     const int rows = min(RU, p.R - rc * RU);
     const int r = blockIdx.x * COMBINE_ROWS + warp;
     __shared__ int red_i[COMBINE_ROWS];
-    // the attention kernel's schedule: all tiles, those before sequence b, b's own
+    // the attention kernel's schedule: all positions, those before sequence b,
+    // b's own tiles
     int tot = 0, before = 0, own = 0;
     for (int s = threadIdx.x; s < p.B; s += blockDim.x) {
-        const int t = seq_tiles(p, s);
+        const int t = seq_slots(p, s);
         tot += t;
         before += s < b ? t : 0;
-        own += s == b ? t : 0;
+        own += s == b ? real_tiles(t) : 0;
     }
     tot = block_sum_i(tot, red_i);
     before = block_sum_i(before, red_i);
@@ -838,7 +879,7 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
     if (Tb == 0 || r >= rows) return;
     const int total = ups * tot;
     const int W = (total + p.num_ctas - 1) / p.num_ctas;
-    const int tpre = ups * before + hr * Tb;
+    const int tpre = ups * before + hr * (Tb + UNIT_COST);
     const int first = tpre / W, n = (tpre + Tb - 1) / W - first + 1;
     if (n == 1) return;  // written by the attention kernel
     const int ridx = rc * RU + r;
@@ -995,9 +1036,10 @@ template <int D, int RP>
 static cudaError_t launch_tc(TcParams &P, cudaStream_t stream) {
     // deepest K/V rings, P and query buffering that fit, in order of preference
     // (K, V, P, Q); a single query buffer stalls a unit's first product on its
-    // query load, which costs less than a shallower ring when units are long
-    static const int choices[][4] = {{3, 4, 2, 2}, {2, 4, 2, 2}, {2, 3, 2, 2}, {2, 3, 1, 2}, {2, 2, 2, 2},
-                                     {2, 2, 1, 2}, {2, 2, 1, 1}};
+    // query load, which costs less than a shallower ring, or a single P buffer
+    // (the softmax then waits on every P.V), when units are long
+    static const int choices[][4] = {{3, 4, 2, 2}, {2, 4, 2, 2}, {2, 3, 2, 2}, {2, 3, 2, 1}, {2, 3, 1, 2},
+                                     {2, 2, 2, 2}, {2, 2, 2, 1}, {2, 2, 1, 2}, {2, 2, 1, 1}};
     constexpr int nchoices = sizeof(choices) / sizeof(choices[0]);
     TcLayout L;
     int k = 0;

@@ -109,6 +109,11 @@ SV_DEV int suffix_tiles(const AttnParams &a, int b) {
     const int C = __ldcg(a.ctx_lens + b);
     return (C >= a.N && C <= a.max_blocks * PAGE) ? (C + TILE_KEYS - 1) / TILE_KEYS : 0;
 }
+// Its schedule positions (the tiles plus UNIT_COST per unit).
+SV_DEV int suffix_slots(const AttnParams &a, int b) {
+    const int t = suffix_tiles(a, b);
+    return t > 0 ? t + UNIT_COST : 0;
+}
 
 __global__ void __launch_bounds__(PREP_THREADS) cascade_prep_kernel(const __grid_constant__ PrepParams p) {
     griddep_wait();
@@ -458,14 +463,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             const float l_p = half == 0 ? l_run + lo : lo + l_run;  // the same sum in both halves
             const float m_p = ntiles > 0 ? m_run : PF_M_NONE;
             // split-context schedule of the suffix call (the attention kernel's
-            // rule): the sequences' tile prefix, one copy per warp, in the P
-            // buffers, which the last P V has finished reading
+            // rule): the prefix of the sequences' schedule positions, one copy
+            // per warp, in the P buffers, which the last P V has finished reading
             int *TP = reinterpret_cast<int *>(base + L.off_p) + (warp - PF_WARP_SM0) * (MAX_SEQS + 1);
             {
                 const int per = (a.B + 31) / 32;
                 const int s0 = min(lane * per, a.B), s1 = min(s0 + per, a.B);
                 int loc = 0;
-                for (int b = s0; b < s1; ++b) loc += suffix_tiles(a, b);
+                for (int b = s0; b < s1; ++b) loc += suffix_slots(a, b);
                 int incl = loc;
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -475,7 +480,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                 int run = incl - loc;
                 for (int b = s0; b < s1; ++b) {
                     TP[b] = run;
-                    run += suffix_tiles(a, b);
+                    run += suffix_slots(a, b);
                 }
                 if (lane == 31) TP[a.B] = incl;
                 __syncwarp();
@@ -490,11 +495,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                 const int Nc = a.rows_unit / G;  // whole query rows per row chunk
                 const int rc = mi / Nc;          // row chunk of the unit that holds query row mi
                 ru = (mi - rc * Nc) * G + mj;
-                const int Tb = TP[mb + 1] - TP[mb];
+                const int T1 = TP[mb + 1] - TP[mb];
+                const int Tb = T1 > 0 ? T1 - UNIT_COST : 0;
                 if (Tb > 0) {
                     const int hr = h * a.RC + rc;
                     const int u = mb * ups + hr;
-                    const int tpre = ups * TP[mb] + hr * Tb;
+                    const int tpre = ups * TP[mb] + hr * T1;
                     const int first = tpre / W;
                     n = (tpre + Tb - 1) / W - first + 1;
                     seg = a.ws_partial + (size_t)(u + first) * sf;

@@ -46,6 +46,12 @@ cudaError_t launch_accept(const AcceptParams &p, int rounds, cudaStream_t stream
 // Keys per work tile: the split-context schedule hands out tiles of TILE_KEYS
 // keys of one (sequence, KV head, row chunk) unit.
 constexpr int TILE_KEYS = 128;
+// The split-context schedule charges every unit UNIT_COST tiles on top of its
+// own, for the fixed work of a unit's start and end (its query rows, the first
+// tile's rescale, the read-out of O), so that CTAs that touch many units get
+// fewer tiles. A unit occupies Tb + UNIT_COST positions of the schedule; the
+// last UNIT_COST hold no work.
+constexpr int UNIT_COST = 2;
 constexpr int PAGE = 16;
 constexpr int ROWS_MAX = 96;       // query rows (N*G) one unit carries
 constexpr int MAX_SEQS = 512;
