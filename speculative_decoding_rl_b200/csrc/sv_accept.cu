@@ -121,6 +121,23 @@ SV_DEV void merge_argmax(float &m, int &i, float m2, int i2) {
     if (i2 >= 0 && (i < 0 || m2 > m || (m2 == m && i2 < i))) { m = m2; i = i2; }
 }
 
+// Element arithmetic shared by the statistics, the pass, the walk's test and
+// the draw, so that every kernel computes the same bits for the same weight:
+//   e(x)  = 2^((l(x) - M) c)                        (pweight)
+//   r_0   = e (1/S),  r_i = max(0, r_{i-1} - q_i) (1/Z_i)   (rstart, rstep)
+//   weight after the chain c_1..c_k = max(0, r_{k-1} - q_k)  (rlast)
+// The reciprocals are correctly rounded (one per row or chain entry), the
+// products and differences are rounded once each and never contracted.
+SV_DEV float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;  // results below 2^-126 of the row maximum's weight flush to zero
+}
+SV_DEV float pweight(float l, float M, float c) { return ex2_ftz(__fmul_rn(__fsub_rn(l, M), c)); }
+SV_DEV float rstart(float e, float invS) { return __fmul_rn(e, invS); }
+SV_DEV float rstep(float r, float q, float invZ) { return __fmul_rn(fmaxf(__fsub_rn(r, q), 0.f), invZ); }
+SV_DEV float rlast(float r, float q) { return fmaxf(__fsub_rn(r, q), 0.f); }
+
 // Next child of node v with index > after, or -1.
 SV_DEV int next_child(const AcceptParams &p, int v, int after) {
     for (int c = after + 1; c < p.N; ++c)
@@ -175,18 +192,35 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_stats_kernel(const AcceptP
     float m = -INFINITY, s = 0.f;
     int ai = -1;
     const float c = p.log2e_over_T;
+    if (GREEDY) {
 #pragma unroll
-    for (int k = 0; k < ACC_PER_THREAD; ++k) {
-        if (isnan(e[k]) || e[k] == INFINITY) { flag = 1; e[k] = -INFINITY; }
-        if (GREEDY) {
+        for (int k = 0; k < ACC_PER_THREAD; ++k) {
+            if (isnan(e[k]) || e[k] == INFINITY) { flag = 1; e[k] = -INFINITY; }
             if (e[k] > m) { m = e[k]; ai = index_of(k); }  // strict: the lowest index among equals
-        } else {
-            m = fmaxf(m, e[k]);
         }
-    }
-    if (!GREEDY && m != -INFINITY) {
+    } else {
+        // fmaxf skips NaN; a NaN or +inf entry then shows as a NaN sum (or an
+        // infinite maximum), and only such a thread redoes its entries with
+        // the non-finite ones replaced by -inf
 #pragma unroll
-        for (int k = 0; k < ACC_PER_THREAD; ++k) s += exp2f((e[k] - m) * c);
+        for (int k = 0; k < ACC_PER_THREAD; ++k) m = fmaxf(m, e[k]);
+        if (m > -INFINITY && m < INFINITY) {
+#pragma unroll
+            for (int k = 0; k < ACC_PER_THREAD; ++k) s += pweight(e[k], m, c);
+        }
+        if (!(m > -INFINITY && m < INFINITY) || isnan(s)) {
+            m = -INFINITY;
+            s = 0.f;
+#pragma unroll
+            for (int k = 0; k < ACC_PER_THREAD; ++k) {
+                if (isnan(e[k]) || e[k] == INFINITY) { flag = 1; e[k] = -INFINITY; }
+                m = fmaxf(m, e[k]);
+            }
+            if (m != -INFINITY) {
+#pragma unroll
+                for (int k = 0; k < ACC_PER_THREAD; ++k) s += pweight(e[k], m, c);
+            }
+        }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -218,8 +252,9 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_stats_kernel(const AcceptP
 //   r_i = max(0, r_{i-1} - q_{c_i}) / Z_i   (i < k),
 //   weight = max(0, r_{k-1} - q_{c_k})      (unnormalised; its sum is Z_k).
 // With k = 0 the weight is e (p_v unnormalised). The pass and the draw compute
-// every weight with these same fp32 operations, so they agree bit for bit.
-// ---------------------------------------------------------------------------
+// every weight with the same fp32 operations (pweight, rstart, rstep, rlast:
+// the divisions as products with correctly rounded reciprocals), so they agree
+// bit for bit.
 // ---------------------------------------------------------------------------
 // 3. Per-slice parts of the pending pass of a sequence.
 // ---------------------------------------------------------------------------
@@ -232,7 +267,7 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_pass_kernel(const AcceptPa
     const AccState *st = w.st + b;
     __shared__ int s_mode, s_v, s_k;
     __shared__ float s_M, s_S;
-    __shared__ float s_Z[64];
+    __shared__ float s_Z[64];  // 1/Z_i
     __shared__ const float *s_q[64];
     if (tid == 0) {
         s_mode = __ldcg(&st->mode);
@@ -251,12 +286,12 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_pass_kernel(const AcceptPa
     const int x0 = j * ACC_SLICE;
     const int n = min(ACC_SLICE, p.V - x0);
     if (tid < k) {
-        s_Z[tid] = __ldcg(&st->Z[tid]);
+        s_Z[tid] = __frcp_rn(__ldcg(&st->Z[tid]));  // 1/Z_i (the last entry is unused)
         s_q[tid] = p.q + ((size_t)b * (p.N - 1) + __ldcg(&st->chain[tid]) - 1) * p.V + x0;
     }
     __syncthreads();
     const float *lrow = p.logits + ((size_t)b * p.N + s_v) * p.V + x0;
-    const float M = s_M, Sv = s_S, c = p.log2e_over_T;
+    const float M = s_M, invS = __frcp_rn(s_S), c = p.log2e_over_T;
     float wsum = 0.f, psum = 0.f;
     if (VEC && k <= 1) {
         // p alone, or the chain case (one draft row): 16-byte loads, all of a
@@ -273,21 +308,21 @@ __global__ void __launch_bounds__(ACC_THREADS) accept_pass_kernel(const AcceptPa
         }
 #pragma unroll
         for (int j = 0; j < J; ++j) {
-            const float e0 = exp2f((lv[j].x - M) * c), e1 = exp2f((lv[j].y - M) * c);
-            const float e2 = exp2f((lv[j].z - M) * c), e3 = exp2f((lv[j].w - M) * c);
+            const float e0 = pweight(lv[j].x, M, c), e1 = pweight(lv[j].y, M, c);
+            const float e2 = pweight(lv[j].z, M, c), e3 = pweight(lv[j].w, M, c);
             psum += (e0 + e1) + (e2 + e3);
             if (k)
-                wsum += (fmaxf(e0 / Sv - qv[j].x, 0.f) + fmaxf(e1 / Sv - qv[j].y, 0.f)) +
-                        (fmaxf(e2 / Sv - qv[j].z, 0.f) + fmaxf(e3 / Sv - qv[j].w, 0.f));
+                wsum += (rlast(rstart(e0, invS), qv[j].x) + rlast(rstart(e1, invS), qv[j].y)) +
+                        (rlast(rstart(e2, invS), qv[j].z) + rlast(rstart(e3, invS), qv[j].w));
         }
     } else {
         for (int x = tid; x < n; x += ACC_THREADS) {
-            const float e = exp2f((__ldg(lrow + x) - M) * c);
+            const float e = pweight(__ldg(lrow + x), M, c);
             psum += e;
             if (k) {
-                float r = e / Sv;
-                for (int i = 0; i + 1 < k; ++i) r = fmaxf(r - __ldg(s_q[i] + x), 0.f) / s_Z[i];
-                wsum += fmaxf(r - __ldg(s_q[k - 1] + x), 0.f);
+                float r = rstart(e, invS);
+                for (int i = 0; i + 1 < k; ++i) r = rstep(r, __ldg(s_q[i] + x), s_Z[i]);
+                wsum += rlast(r, __ldg(s_q[k - 1] + x));
             }
         }
     }
@@ -321,10 +356,10 @@ SV_DEV int walk_sampling(const AcceptParams &p, AccState &S, int b) {
             S.flags |= SV_FLAG_BAD_TOKEN;  // counts as a rejection
         } else {
             const float u = philox_uniform(key, (uint32_t)b, (uint32_t)ch, 0u);
-            float r = exp2f((S.Ld[ch] - S.rowM[v]) * c) / S.rowS[v];
+            float r = rstart(pweight(S.Ld[ch], S.rowM[v], c), __frcp_rn(S.rowS[v]));
             for (int i = 0; i < S.nchain; ++i) {
                 const float qx = __ldg(p.q + ((size_t)b * (p.N - 1) + S.chain[i] - 1) * p.V + d);
-                r = fmaxf(r - qx, 0.f) / S.Z[i];
+                r = rstep(r, qx, __frcp_rn(S.Z[i]));
             }
             acc = u * S.Qd[ch] < r;
         }
@@ -502,7 +537,7 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
         // the drawn slice's weights, with the pass's arithmetic, staged in shared
         // memory; a thread's loads are all in flight before the first is used
         const float *lrow = p.logits + ((size_t)b * N + v) * p.V + x0;
-        const float M = S.rowM[v], Sv = S.rowS[v];
+        const float M = S.rowM[v], invS = __frcp_rn(S.rowS[v]);
         auto put = [&](int x, float wgt) { wbuf[x + (x >> 5)] = wgt; };
         if (p.vec && k <= 1) {
             const float4 *l4 = reinterpret_cast<const float4 *>(lrow);
@@ -525,20 +560,20 @@ __global__ void __launch_bounds__(WALK_THREADS, 1) accept_walk_kernel(const Acce
                 const float q[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float ex = exp2f((l[e] - M) * c);
-                    put(4 * i + e, k ? fmaxf(ex / Sv - q[e], 0.f) : ex);
+                    const float ex = pweight(l[e], M, c);
+                    put(4 * i + e, k ? rlast(rstart(ex, invS), q[e]) : ex);
                 }
             }
         } else {
             for (int x = tid; x < n; x += WALK_THREADS) {
-                const float e = exp2f((__ldg(lrow + x) - M) * c);
+                const float e = pweight(__ldg(lrow + x), M, c);
                 float wgt = e;
                 if (use_w) {
-                    float r = e / Sv;
+                    float r = rstart(e, invS);
                     for (int i = 0; i + 1 < k; ++i)
-                        r = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[i] - 1) * p.V + x0 + x), 0.f) /
-                            S.Z[i];
-                    wgt = fmaxf(r - __ldg(p.q + ((size_t)b * (N - 1) + S.chain[k - 1] - 1) * p.V + x0 + x), 0.f);
+                        r = rstep(r, __ldg(p.q + ((size_t)b * (N - 1) + S.chain[i] - 1) * p.V + x0 + x),
+                                  __frcp_rn(S.Z[i]));
+                    wgt = rlast(r, __ldg(p.q + ((size_t)b * (N - 1) + S.chain[k - 1] - 1) * p.V + x0 + x));
                 }
                 put(x, wgt);
             }
