@@ -344,6 +344,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             uint8_t *ring = base + (is_k ? L.off_k : 0u);
             const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
             int lu = -1, issued_tiles = 0;
+            int rs = 0;  // ring slot of tile lt, and its phase
+            uint32_t rph = 0;
             TileInfo ti = t_first;
             for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
                 const int h = ti.hr / p.RC, rc = ti.hr - h * p.RC;
@@ -365,8 +367,9 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         tma_load_3d(qdst + a * RP * 128, &P.tm_q, &q_full[qb], a * 64, h * p.G,
                                     ti.b * p.N + rc * P.Nc);
                 }
-                const int s = lt % NR;
-                if (!mbar_wait(&empty[s], ((lt / NR) & 1) ^ 1, abort_flag, p.wait_limit_ns)) break;
+                const int s = rs;
+                if (!mbar_wait(&empty[s], rph ^ 1u, abort_flag, p.wait_limit_ns)) break;
+                if (++rs == NR) { rs = 0; rph ^= 1u; }
                 mbar_arrive_expect_tx(&full[s], L.tile_bytes);
                 uint8_t *dst = ring + s * L.tile_bytes;
 #pragma unroll
@@ -417,9 +420,12 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
         // is released to its PV through vz, after its V has landed, so this warp
         // stays within one phase of the V ring.
         TileInfo ti = t_first;
+        int vs = 0;  // V slot of tile lt, and its phase
+        uint32_t vph = 0;
         for (int lt = 0; lt < ntiles; ++lt, next_tile(ti, TP, p.B, ups)) {
-            const int s = lt % NV;
-            const uint32_t par = (lt / NV) & 1;
+            const int s = vs;
+            const uint32_t par = vph;
+            if (++vs == NV) { vs = 0; vph ^= 1u; }
             const bool landed = mbar_test(&v_full[s], par) || mbar_wait(&v_full[s], par, abort_flag, p.wait_limit_ns);
             if (!__all_sync(0xffffffffu, landed)) break;
             // keys [k0, k1) of the tile: past ctx_len but inside its last page (pages
@@ -448,6 +454,10 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             constexpr uint32_t idq = idesc_bf16(128, RP, false, false);
             constexpr uint32_t idp = idesc_bf16(128, RP, true, true);
             int nq = 0, np = 0, lu = -1, qb = 0, lup = -1;
+            // ring slots of tiles nq (K) and np (V, P) and their phases, advanced
+            // by one per product (no division by the runtime ring sizes)
+            int ks = 0, vs = 0, ps = 0;
+            uint32_t kph = 0, vph = 0, pph = 0;
             TileInfo tq = t_first;
             TileInfo tp = tq;
             uint32_t idle = 0;
@@ -458,9 +468,9 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     const bool newu = (nq == 0 || tq.j == 0);
                     const int lu_n = newu ? lu + 1 : lu;
                     const int qb_n = qbuf(lu_n);
-                    const int s = nq % NK, sb = nq & 1;
+                    const int s = ks, sb = nq & 1;
                     if ((!newu || mbar_test(&q_full[qb_n], qphase(lu_n))) &&
-                        mbar_test(&k_full[s], (nq / NK) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
+                        mbar_test(&k_full[s], kph) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
                         lu = lu_n;
                         qb = qb_n;
                         tc_fence_after();
@@ -475,6 +485,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         mma_commit(&s_full[sb]);
                         mma_commit(&k_empty[s]);
                         if (nq == ntiles - 1 || tq.j == tq.Tb - 1) mma_commit(&q_empty[qb]);
+                        if (++ks == NK) { ks = 0; kph ^= 1u; }
                         ++nq;
                         if (nq < ntiles) next_tile(tq, TP, p.B, ups);
                         progressed = true;
@@ -483,9 +494,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 if (np < nq) {
                     const bool newu = (np == 0 || tp.j == 0);
                     const int lup_n = newu ? lup + 1 : lup;
-                    const int s = np % NV, pb = np % NP, ob = lup_n & 1;
-                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&v_full[s], (np / NV) & 1) &&
-                        mbar_test(&vz[s], (np / NV) & 1) &&
+                    const int s = vs, pb = ps, ob = lup_n & 1;
+                    if (mbar_test(&p_full[pb], pph) && mbar_test(&v_full[s], vph) && mbar_test(&vz[s], vph) &&
                         (!newu || mbar_test(&o_free[ob], ((lup_n >> 1) & 1) ^ 1))) {
                         lup = lup_n;
                         tc_fence_after();
@@ -500,6 +510,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         mma_commit(&o_full[np & 1]);
                         mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[s]);
+                        if (++vs == NV) { vs = 0; vph ^= 1u; }
+                        if (++ps == NP) { ps = 0; pph ^= 1u; }
                         ++np;
                         if (np < ntiles) next_tile(tp, TP, p.B, ups);
                         progressed = true;
@@ -641,6 +653,8 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
 
         // one pass past the last tile closes and finishes the CTA's last unit
         TileInfo tnext = t_first;
+        int pslot = 0;  // P buffer of tile lt, and its phase
+        uint32_t pphase = 0;
         for (int lt = 0; lt <= ntiles && ok; ++lt) {
             const bool end = lt == ntiles;
             const TileInfo ti = end ? TileInfo{0, 0, 0, 1} : tnext;
@@ -801,8 +815,9 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 packed[c4 * 2] = *reinterpret_cast<uint32_t *>(&h0);
                 packed[c4 * 2 + 1] = *reinterpret_cast<uint32_t *>(&h1);
             }
-            const int pb = lt % NP;
-            if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
+            const int pb = pslot;
+            if (!(ok = wait_w(&p_empty[pb], pphase ^ 1u))) break;
+            if (++pslot == NP) { pslot = 0; pphase ^= 1u; }
             uint8_t *pbuf = base + L.off_p + pb * L.p_bytes;
 #pragma unroll
             for (int c8 = 0; c8 < CW / 8; ++c8) {
