@@ -141,7 +141,7 @@ class ClockSampler:
         return False
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
+        sm, mx, pw, reasons = [], [], [], set()
         for line in (self.out or "").splitlines():
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -151,6 +151,10 @@ class ClockSampler:
                 mx.append(float(parts[2]))
             except ValueError:
                 continue
+            try:
+                pw.append(float(parts[3]))
+            except ValueError:
+                pass
             names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
             for n, v in zip(names, parts[5:9]):
                 if v.lower() == "active":
@@ -158,7 +162,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "power_w": statistics.median(pw) if pw else None, "samples": len(sm)}
 
 
 def dist_setup():

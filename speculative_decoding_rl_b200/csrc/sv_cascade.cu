@@ -234,6 +234,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
         if (lane == 0) {
             const int32_t *bt = p.block_table + (size_t)b0 * a.max_blocks;  // the group's pages
             int issued_k = 0, issued_v = 0;
+            int sk = 0, sv = 0;  // ring slots of tile lt and their phases (no runtime division)
+            uint32_t kph = 0, vph = 0;
             for (int lt = 0; lt < ntiles; ++lt) {
                 int blks[PF_KEYS / PAGE];
 #pragma unroll
@@ -242,8 +244,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     const int blk = page * PAGE < P ? __ldg(bt + page) : -1;
                     blks[pg] = (blk >= 0 && blk < a.num_blocks) ? blk : a.num_blocks;  // past the pool: zeros
                 }
-                const int sk = lt % NK;
-                if (!mbar_wait(&k_empty[sk], ((lt / NK) & 1) ^ 1, abort_flag, a.wait_limit_ns)) break;
+                if (!mbar_wait(&k_empty[sk], kph ^ 1u, abort_flag, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&k_full[sk], L.tile);
                 uint8_t *kd = base + L.off_k + sk * L.tile;
 #pragma unroll
@@ -251,8 +252,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     for (int q = 0; q < nDA; ++q)
                         tma_load_4d(kd + q * PF_ATOM + pg * 2048, &p.tm_k, &k_full[sk], q * 64, 0, h, blks[pg]);
                 issued_k = lt + 1;
-                const int sv = lt % NV;
-                if (!mbar_wait(&v_empty[sv], ((lt / NV) & 1) ^ 1, abort_flag, a.wait_limit_ns)) break;
+                if (++sk == NK) { sk = 0; kph ^= 1u; }
+                if (!mbar_wait(&v_empty[sv], vph ^ 1u, abort_flag, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&v_full[sv], L.tile);
                 uint8_t *vd = base + L.off_v + sv * L.tile;
 #pragma unroll
@@ -260,6 +261,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     for (int q = 0; q < nDA; ++q)
                         tma_load_4d(vd + q * PF_ATOM + pg * 2048, &p.tm_v, &v_full[sv], q * 64, 0, h, blks[pg]);
                 issued_v = lt + 1;
+                if (++sv == NV) { sv = 0; vph ^= 1u; }
             }
             if (*abort_flag) {
                 // this CTA's own copies land before it can exit
@@ -277,13 +279,15 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             const uint32_t qa = smem_u32(base + L.off_q);
             bool ok = mbar_wait(q_ready, 0, abort_flag, a.wait_limit_ns);
             int nq = 0, np = 0;
+            int ks = 0, vs = 0, ps = 0;  // ring slots of tiles nq (K) and np (V, P) and their phases
+            uint32_t kph = 0, vph = 0, pph = 0;
             uint32_t idle = 0;
             uint64_t idle_since = 0;
             while (ok && np < ntiles) {
                 bool progressed = false;
                 if (nq < ntiles) {
-                    const int sk = nq % NK, sb = nq & 1;
-                    if (mbar_test(&k_full[sk], (nq / NK) & 1) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
+                    const int sk = ks, sb = nq & 1;
+                    if (mbar_test(&k_full[sk], kph) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
                         tc_fence_after();
                         const uint32_t ka = smem_u32(base + L.off_k + sk * L.tile);
 #pragma unroll
@@ -294,13 +298,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                         }
                         mma_commit(&s_full[sb]);
                         mma_commit(&k_empty[sk]);
+                        if (++ks == NK) { ks = 0; kph ^= 1u; }
                         ++nq;
                         progressed = true;
                     }
                 }
                 if (np < nq) {
-                    const int sv = np % NV, pb = np % NP;
-                    if (mbar_test(&p_full[pb], (np / NP) & 1) && mbar_test(&v_full[sv], (np / NV) & 1)) {
+                    const int sv = vs, pb = ps;
+                    if (mbar_test(&p_full[pb], pph) && mbar_test(&v_full[sv], vph)) {
                         tc_fence_after();
                         const uint32_t va = smem_u32(base + L.off_v + sv * L.tile);
                         const uint32_t pa = smem_u32(base + L.off_p + pb * 2 * PF_ATOM);
@@ -313,6 +318,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                         mma_commit(&o_full[np & 1]);
                         mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[sv]);
+                        if (++vs == NV) { vs = 0; vph ^= 1u; }
+                        if (++ps == NP) { ps = 0; pph ^= 1u; }
                         ++np;
                         progressed = true;
                     }
@@ -379,8 +386,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
         const float sc = a.scale_log2;
         float m_run = PF_M_NONE, l_run = 0.f;  // l_run: this half's keys only
         bool ok = true;
+        int pslot = 0;  // P buffer of tile lt, and its phase
+        uint32_t pphase = 0;
         for (int lt = 0; lt < ntiles && ok; ++lt) {
-            const int sb = lt & 1, pb = lt % NP;
+            const int sb = lt & 1, pb = pslot;
             const int valid = P - lt * PF_KEYS - half * 64;  // keys of this half inside the prefix
             if (!(ok = wait_w(&s_full[sb], (lt >> 1) & 1))) break;
             tc_fence_after();
@@ -424,7 +433,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                 tmem_wait_st();
             }
             m_run = m_new;
-            if (!(ok = wait_w(&p_empty[pb], ((lt / NP) & 1) ^ 1))) break;
+            if (!(ok = wait_w(&p_empty[pb], pphase ^ 1u))) break;
+            if (++pslot == NP) { pslot = 0; pphase ^= 1u; }
             uint8_t *pt = base + L.off_p + pb * 2 * PF_ATOM;
 #pragma unroll
             for (int c0 = 0; c0 < 64; c0 += 32) {

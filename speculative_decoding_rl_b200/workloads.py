@@ -352,6 +352,18 @@ def workload(name: str, **over) -> Workload:
         acc = dict(num_seqs=64, num_rows=N, vocab=128256, seed=2005, logit_std=3.0,
                    draft_noise=0.6, temperature=T, draft_temperature=0.7)
         w = Workload(f"{name}_T{T:g}", 32, attn, acc)
+    elif name == "grpo_long_prompt":
+        # the same group shape with long prompts: 8 groups of 16 rollouts whose
+        # 8192 shared prompt tokens are most of each context (the shared pages,
+        # 268 MB a layer, no longer fit in L2)
+        N = 7
+        T = over.pop("temperature", 0.0)
+        attn = dict(num_q_rows=N, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                    ctx=dict(kind="uniform", lo=8192 + 512, hi=8192 + 4096), num_seqs=128,
+                    seed=1006, shared_prefix_groups=8, shared_prefix_tokens=8192)
+        acc = dict(num_seqs=128, num_rows=N, vocab=128256, seed=2006, logit_std=3.0,
+                   draft_noise=0.6, temperature=T, draft_temperature=0.7)
+        w = Workload(f"{name}_T{T:g}", 32, attn, acc)
     else:
         raise ValueError(f"unknown workload {name}")
     for k, v in over.items():

@@ -124,8 +124,9 @@ def test_invalid_members_and_bad_prefix_pages():
     assert_attention_close(got[0], want[0], "valid member beside invalid ones")
 
 
-def test_grpo_full_size_sampled_rows():
-    w = W.workload("grpo_shared_prefix")
+@pytest.mark.parametrize("name", ["grpo_shared_prefix", "grpo_long_prompt"])
+def test_grpo_full_size_sampled_rows(name):
+    w = W.workload(name)
     a = W.build_attention(w)
     got, st = run(a, a.group_offsets, a.prefix_lens)
     assert (st == 0).all()
@@ -134,5 +135,5 @@ def test_grpo_full_size_sampled_rows():
                      rng.integers(0, a.num_q_heads, 64)], axis=1).astype(np.int32)
     want = oracle.cascade_attention(a, a.group_offsets, a.prefix_lens, rows=rows)
     sel = got[rows[:, 0], rows[:, 1], rows[:, 2]]
-    max_abs, mean_rel = assert_attention_close(sel, want, "grpo full size, sampled rows")
-    print(f"grpo full size: max_abs {max_abs:.2e} mean_rel {mean_rel:.2e}")
+    max_abs, mean_rel = assert_attention_close(sel, want, f"{name} full size, sampled rows")
+    print(f"{name} full size: max_abs {max_abs:.2e} mean_rel {mean_rel:.2e}")

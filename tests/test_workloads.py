@@ -66,3 +66,20 @@ def test_draft_recipe_gives_about_seventy_percent_acceptance():
     assert 0.6 < float(beta.mean()) < 0.8
     # drafts are valid tokens drawn from q
     assert int(a.draft_tokens.min()) >= 0 and int(a.draft_tokens.max()) < a.vocab
+
+
+def test_long_prompt_groups_share_their_prompt_pages():
+    w = W.workload("grpo_long_prompt")
+    a = W.build_attention(w)
+    tbl = a.block_table.numpy()
+    assert a.num_seqs == 128 and list(a.group_offsets) == list(range(0, 129, 16))
+    assert list(a.prefix_lens) == [8192] * 8
+    npg = 8192 // 16
+    for g in range(8):
+        rows = tbl[g * 16:(g + 1) * 16, :npg]
+        assert (rows == rows[0]).all()
+        # each member's own pages follow the prompt and are its alone
+        own = [set(tbl[b, npg:(int(a.ctx_lens[b]) + 15) // 16]) for b in range(g * 16, (g + 1) * 16)]
+        assert all(len(x & y) == 0 for i, x in enumerate(own) for y in own[i + 1:])
+    lens = a.ctx_lens.numpy()
+    assert lens.min() >= 8192 + 512 and lens.max() <= 8192 + 4096
