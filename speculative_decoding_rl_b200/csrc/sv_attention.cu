@@ -260,6 +260,12 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
     uint64_t *done_bar = o_free + 2;
     uint64_t *wg_bar = done_bar + 1;   // [NWG] warpgroup-local barriers
     uint64_t *vz = wg_bar + NWG;       // [NV] the tile's V is ready for its PV (rows past ctx_len zeroed)
+    // With a two-slot K ring, tile t's K slot is its S buffer t & 1 and the QK
+    // product that frees the slot is the one s_full[t & 1] marks: the K producer
+    // waits on s_full. Likewise with two P buffers, buffer t & 1 is freed by
+    // tile t's PV, which o_full[t & 1] marks. One commit fewer per tile each.
+    uint64_t *k_free = NK == 2 ? s_full : k_empty;
+    uint64_t *p_free = NP == 2 ? o_full : p_empty;
     int *TP = reinterpret_cast<int *>(base + L.off_tp);
     int *CL = reinterpret_cast<int *>(base + L.off_cl);
     float *red = reinterpret_cast<float *>(base + L.off_red);
@@ -339,7 +345,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             const bool is_k = warp == WARP_K;
             const int NR = is_k ? NK : NV;
             uint64_t *full = is_k ? k_full : v_full;
-            uint64_t *empty = is_k ? k_empty : v_empty;
+            uint64_t *empty = is_k ? k_free : v_empty;
             const CUtensorMap *tm = is_k ? &P.tm_k : &P.tm_v;
             uint8_t *ring = base + (is_k ? L.off_k : 0u);
             const uint32_t q_box_bytes = 64u * p.G * P.Nc * 2u;
@@ -458,6 +464,13 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
             // by one per product (no division by the runtime ring sizes)
             int ks = 0, vs = 0, ps = 0;
             uint32_t kph = 0, vph = 0, pph = 0;
+            // operand descriptors of the ring bases; a product adds its stage's
+            // offset (in 16-byte units; shared addresses stay below 2^18 bytes,
+            // so the 14-bit address field does not carry)
+            const uint64_t kdesc = sw128_desc(smem_u32(base + L.off_k), 16, 1024);
+            const uint64_t qdesc = sw128_desc(smem_u32(base + L.off_q), 16, 1024);
+            const uint64_t vdesc = sw128_desc(smem_u32(base), ATOM, 1024);
+            const uint64_t pdesc = sw128_desc(smem_u32(base + L.off_p), ATOM, 1024);
             TileInfo tq = t_first;
             TileInfo tp = tq;
             uint32_t idle = 0;
@@ -474,16 +487,16 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                         lu = lu_n;
                         qb = qb_n;
                         tc_fence_after();
-                        const uint32_t ka = smem_u32(base + L.off_k + s * L.tile_bytes);
-                        const uint32_t qa = smem_u32(base + L.off_q + qb * L.q_bytes);
+                        const uint64_t ka = kdesc + ((s * L.tile_bytes) >> 4);
+                        const uint64_t qa = qdesc + ((qb * L.q_bytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(ka + (kk >> 2) * ATOM + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(qa + (kk >> 2) * (RP * 128) + (kk & 3) * 32, 16, 1024);
+                            const uint64_t ad = ka + (((kk >> 2) * ATOM + (kk & 3) * 32) >> 4);
+                            const uint64_t bd = qa + (((kk >> 2) * (RP * 128) + (kk & 3) * 32) >> 4);
                             mma_bf16_ss(tmem + sb * RPa, ad, bd, idq, kk > 0);
                         }
                         mma_commit(&s_full[sb]);
-                        mma_commit(&k_empty[s]);
+                        if (NK != 2) mma_commit(&k_empty[s]);
                         if (nq == ntiles - 1 || tq.j == tq.Tb - 1) mma_commit(&q_empty[qb]);
                         if (++ks == NK) { ks = 0; kph ^= 1u; }
                         ++nq;
@@ -495,20 +508,22 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                     const bool newu = (np == 0 || tp.j == 0);
                     const int lup_n = newu ? lup + 1 : lup;
                     const int s = vs, pb = ps, ob = lup_n & 1;
-                    if (mbar_test(&p_full[pb], pph) && mbar_test(&v_full[s], vph) && mbar_test(&vz[s], vph) &&
+                    // vz follows v_full: the status warp arrives on it after it has
+                    // seen the tile's V land
+                    if (mbar_test(&p_full[pb], pph) && mbar_test(&vz[s], vph) &&
                         (!newu || mbar_test(&o_free[ob], ((lup_n >> 1) & 1) ^ 1))) {
                         lup = lup_n;
                         tc_fence_after();
-                        const uint32_t va = smem_u32(base + s * L.tile_bytes);
-                        const uint32_t pa = smem_u32(base + L.off_p + pb * L.p_bytes);
+                        const uint64_t va = vdesc + ((s * L.tile_bytes) >> 4);
+                        const uint64_t pa = pdesc + ((pb * L.p_bytes) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < TILE_KEYS / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(va + kk * 2048, ATOM, 1024);
-                            const uint64_t bd = sw128_desc(pa + kk * 2048, ATOM, 1024);
+                            const uint64_t ad = va + ((kk * 2048) >> 4);
+                            const uint64_t bd = pa + ((kk * 2048) >> 4);
                             mma_bf16_ss(tmem + (2 + ob) * RPa, ad, bd, idp, (kk > 0 || !newu) ? 1u : 0u);
                         }
                         mma_commit(&o_full[np & 1]);
-                        mma_commit(&p_empty[pb]);
+                        if (NP != 2) mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[s]);
                         if (++vs == NV) { vs = 0; vph ^= 1u; }
                         if (++ps == NP) { ps = 0; pph ^= 1u; }
@@ -816,7 +831,7 @@ __global__ void __launch_bounds__(tc_threads(RP), 1) attn_tc_kernel(const __grid
                 packed[c4 * 2 + 1] = *reinterpret_cast<uint32_t *>(&h1);
             }
             const int pb = pslot;
-            if (!(ok = wait_w(&p_empty[pb], pphase ^ 1u))) break;
+            if (!(ok = wait_w(&p_free[pb], pphase ^ 1u))) break;
             if (++pslot == NP) { pslot = 0; pphase ^= 1u; }
             uint8_t *pbuf = base + L.off_p + pb * L.p_bytes;
 #pragma unroll
