@@ -388,36 +388,59 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
         bool ok = true;
         int pslot = 0;  // P buffer of tile lt, and its phase
         uint32_t pphase = 0;
+        // One pass over this half's 64 scores of a tile: their maximum, and p =
+        // 2^(s scale - m) against a given maximum, packed as bf16 pairs, with
+        // their sum. Keys past the prefix get p = 0.
+        auto scores_to_p = [&](uint32_t sa, int valid, float m, float &mx, float &tsum, uint32_t *pk) {
+            mx = -INFINITY;
+            tsum = 0.f;
+#pragma unroll
+            for (int c0 = 0; c0 < 64; c0 += 32) {
+                float v[32];
+                tmem_ld32(sa + c0, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    float v0 = v[c], v1 = v[c + 1];
+                    if (valid < 64) {
+                        v0 = c0 + c < valid ? v0 : -INFINITY;
+                        v1 = c0 + c + 1 < valid ? v1 : -INFINITY;
+                    }
+                    mx = fmaxf(mx, fmaxf(v0, v1));
+                    const float p0 = ex2_approx(fmaf(v0, sc, -m)), p1 = ex2_approx(fmaf(v1, sc, -m));
+                    tsum += p0 + p1;
+                    const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
+                    pk[(c0 + c) >> 1] = *reinterpret_cast<const uint32_t *>(&hv);
+                }
+            }
+        };
         for (int lt = 0; lt < ntiles && ok; ++lt) {
             const int sb = lt & 1, pb = pslot;
             const int valid = P - lt * PF_KEYS - half * 64;  // keys of this half inside the prefix
             if (!(ok = wait_w(&s_full[sb], (lt >> 1) & 1))) break;
             tc_fence_after();
             const uint32_t sa = lane_base + COL_S + sb * PF_KEYS + half * 64;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                float v[32];
-                tmem_ld32(sa + c0, v);
-                tmem_wait_ld();
-                if (valid >= 64) {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, v[c]);
-                } else {
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) mx = fmaxf(mx, c0 + c < valid ? v[c] : -INFINITY);
-                }
-            }
+            // p against the running maximum, which stays unless this tile raises
+            // it: a row's first tile, or a score above it by more than 2^8 (rare
+            // after the first tile); a raise reads the scores once more
+            float mx, tsum;
+            uint32_t pk[32];
+            scores_to_p(sa, valid, m_run, mx, tsum, pk);
             mx = fmaxf(mx, swap(mx, lt & 1, ok));
             if (!ok) break;
-            // the running max is raised on a row's first tile, or when a score
-            // beats it by more than 2^8; otherwise the tile folds in as it is
             const float cand = mx * sc;
             const bool raise = m_run == PF_M_NONE || cand > m_run + PF_RESCALE_LOG2;
             const float m_new = raise ? fmaxf(m_run, cand) : m_run;
+            const bool wraise = __any_sync(0xffffffffu, raise);
+            if (wraise) {
+                float mx2;
+                scores_to_p(sa, valid, m_new, mx2, tsum, pk);
+            }
+            tc_fence_before();
+            warp_arrive(&s_empty[sb]);  // this tile's scores are read
             const float alpha = ex2_approx(m_run - m_new);  // first tile: 0; unchanged: 1
-            l_run *= alpha;
-            if (lt > 0 && __any_sync(0xffffffffu, raise)) {
+            l_run = l_run * alpha + tsum;
+            if (lt > 0 && wraise) {
                 // this half's dims of O, once the previous tile's P V has landed
                 if (!(ok = wait_w(&o_full[(lt - 1) & 1], ((lt - 1) >> 1) & 1))) break;
                 tc_fence_after();
@@ -437,30 +460,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
             if (++pslot == NP) { pslot = 0; pphase ^= 1u; }
             uint8_t *pt = base + L.off_p + pb * 2 * PF_ATOM;
 #pragma unroll
-            for (int c0 = 0; c0 < 64; c0 += 32) {
-                float v[32];
-                tmem_ld32(sa + c0, v);
-                tmem_wait_ld();
-                uint32_t pk[16];
-#pragma unroll
-                for (int c = 0; c < 32; c += 2) {
-                    float p0 = ex2_approx(fmaf(v[c], sc, -m_run));
-                    float p1 = ex2_approx(fmaf(v[c + 1], sc, -m_run));
-                    if (valid < 64) {
-                        p0 = c0 + c < valid ? p0 : 0.f;
-                        p1 = c0 + c + 1 < valid ? p1 : 0.f;
-                    }
-                    l_run += p0 + p1;
-                    const __nv_bfloat162 hv = __floats2bfloat162_rn(p0, p1);
-                    pk[c >> 1] = *reinterpret_cast<const uint32_t *>(&hv);
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4)
-                    *reinterpret_cast<uint4 *>(pt + kmajor_off(ell, half * 8 + (c0 >> 3) + q4)) =
-                        make_uint4(pk[4 * q4], pk[4 * q4 + 1], pk[4 * q4 + 2], pk[4 * q4 + 3]);
-            }
+            for (int q = 0; q < 8; ++q)
+                *reinterpret_cast<uint4 *>(pt + kmajor_off(ell, half * 8 + q)) =
+                    make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             tc_fence_before();
-            warp_arrive(&s_empty[sb]);
             fence_proxy_async_smem();
             warp_arrive(&p_full[pb]);
         }

@@ -235,9 +235,15 @@ SV_DEV void tmem_st16(uint32_t taddr, const float *v) {
 SV_DEV void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // One column: 32 lanes x 32 bits (one value per thread of the warp).
+// One column, waited for in the same asm block: the register is valid on return.
 SV_DEV float tmem_ld1(uint32_t taddr) {
     uint32_t r;
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r)
+        : "r"(taddr)
+        : "memory");
     return __uint_as_float(r);
 }
 SV_DEV void tmem_st1(uint32_t taddr, float v) {
