@@ -12,27 +12,37 @@
 //           G query heads that read KV head h; a chunk holds whole query rows
 //           i, at most ROWS_MAX rows (i, g) in all;
 //   tile  = TILE_KEYS consecutive keys of one unit;
-//   all tiles of all units are laid end to end and cut into num_ctas equal
-//   ranges, so every SM streams the same number of KV bytes whatever the mix
-//   of context lengths. A CTA writes one partial (unnormalised O, running max
-//   m, running sum l; log2 domain) per unit it touches to workspace slot
-//   unit + cta, unique because consecutive units share at most one CTA; the
-//   combine kernel merges a unit's partials by their log-sum-exp.
+//   all tiles of all units are laid end to end, each unit followed by
+//   UNIT_COST empty positions for its fixed cost, and the positions are cut
+//   into num_ctas equal ranges, so every SM carries the same load whatever the
+//   mix of context lengths. A CTA writes one partial (unnormalised O, running
+//   max m, running sum l; log2 domain) per unit it touches but does not cover
+//   whole to workspace slot unit + cta, unique because consecutive units share
+//   at most one CTA; the combine kernel merges a unit's partials by their
+//   log-sum-exp. A unit one CTA covers whole is written out directly.
 //
-// Inside a CTA (warp-specialised, tcgen05 + TMA, sm_100a):
-//   warp 0       TMA producer: per tile, 8 pages x {K, V} x (D/64) boxes of
-//                16 keys x 64 dims into a 128B-swizzled stage, plus the unit's
-//                query rows (one 3-D box per 64 dims) when a unit starts;
-//   warp 1       TMEM allocator and MMA issuer: S^T = K Q^T (M = 128 keys,
-//                N = padded rows RP, K = D) and O^T = V^T P^T (M = 128 dims,
+// Inside a CTA (warp-specialised, tcgen05 + TMA, sm_100a), with MATH_WARPS =
+// 4 x the number of softmax warpgroups:
+//   warps 0 .. MATH_WARPS-1  softmax warpgroups, each owning CW of the RP row
+//                columns; warp w owns TMEM lane quadrant w % 4 (a key for S, a
+//                head dim for O). Per tile: load S, mask, a warpgroup vote on
+//                raising the running column maxima (rare after a unit's first
+//                tile; then the maxima are reduced over the 128 keys and O^T in
+//                TMEM is rescaled), p = 2^(s scale - m) as bf16 into a swizzled
+//                shared tile for the PV product;
+//   WARP_K       TMA producer of the query rows (one 3-D box per 64 dims when a
+//                unit starts) and of K: per tile, 8 pages x (D/64) boxes of 16
+//                keys x 64 dims into a 128B-swizzled ring slot;
+//   WARP_MMA     TMEM allocator and MMA issuer: S^T = K Q^T (M = 128 keys,
+//                N = padded rows RP, K = D) and O^T += V^T P^T (M = 128 dims,
 //                N = RP, K = 128 keys), fp32 accumulators in TMEM, S and O
-//                double-buffered;
-//   warps 2-9    two warpgroups, each owning half of the RP row columns: each
-//                thread owns one TMEM lane (a key for S, a head dim for O).
-//                Per tile: load S, mask, column max over the 128 keys (warp
-//                max + shared memory), online-softmax update, P (bf16) into a
-//                swizzled shared tile for the PV MMA, then rescale-and-add the
-//                previous tile's O^T into register accumulators.
+//                double-buffered; it polls both queues and issues whichever
+//                product is ready;
+//   WARP_V       TMA producer of V, as for K;
+//   WARP_ST      per-sequence status flags (and zero output for invalid
+//                sequences), then the V ring: the rows of keys past ctx_len in
+//                a tile's last page are zeroed before the tile goes to its PV.
+// Ring slots and barrier phases are counters advanced once per tile.
 // Putting keys on the MMA M dimension keeps the tensor-core work at
 // 2 * 128 * RP * D per tile however few rows N*G there are, instead of
 // padding the rows to 128.
