@@ -613,8 +613,10 @@ def run_ours(args, world, rank, local):
         e2.record(stream)
         torch.cuda.synchronize()
         e2e_elapsed = max_over_ranks(s2.elapsed_time(e2) / 1e3, world)
+        # e2e step k ran with Philox seed k on the same inputs as device step k
+        e2e_same = bool(np.array_equal(res_len.numpy(), lens_out[:K].cpu().numpy()))
         e2e = {"value": steps_total / e2e_elapsed, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h),
+               "d2h_bytes_per_step": int(d2h), "accept_len_matches_device": e2e_same,
                "copied": "every layer's q, logits, draft probs, drafts, block table, ctx_lens in; accept_len, "
                          "next_token out; the KV cache is the model's resident state and is not copied",
                "overlap": "copies on a second stream, each layer waiting for its own q and the accept for "
