@@ -202,7 +202,10 @@ SV_API sv_status sv_cascade_verify_attention(const sv_attn_desc *desc, const sv_
  * Philox4x32-10 with key {seed_lo32, seed_hi32} and counter {b, c, tag, 0}
  * (Salmon et al., SC'11). InvCDF(w, u) is the smallest x with
  * sum_{y<=x} w(y) > u * sum(w), else the last x with w(x) > 0.
- * Arithmetic is fp32. A sequence flagged SV_FLAG_NONFINITE gets
+ * Arithmetic is fp32: 2^x by the hardware approximation, divisions by a row's
+ * or a residual's mass as products with its correctly rounded reciprocal, sums
+ * in a fixed order, so a call's results depend only on its inputs and seed.
+ * A sequence flagged SV_FLAG_NONFINITE gets
  * accept_len 0, next_token 0; a bad draft token counts as rejected.
  * The work is spread over every SM: one pass reads every logit once for the
  * row statistics, a per-sequence walk takes the decisions, and each rejection
