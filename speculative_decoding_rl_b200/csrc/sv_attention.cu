@@ -1106,7 +1106,6 @@ static cudaError_t launch_tc_rp(TcParams &P, int RP, cudaStream_t stream) {
         case 32: return launch_tc<D, 32>(P, stream);
         case 48: return launch_tc<D, 48>(P, stream);
         case 64: return launch_tc<D, 64>(P, stream);
-        case 80: return launch_tc<D, 80>(P, stream);
         case 96: return launch_tc<D, 96>(P, stream);
     }
     return cudaErrorInvalidValue;
@@ -1123,7 +1122,9 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
         !encode_pool_map(&P.tm_v, p.v_pool, p.num_blocks, p.Hkv, p.D) ||
         !encode_q_map(&P.tm_q, p.q, p.B, p.N, p.Hq, p.D, p.G, Nc))
         return cudaErrorInvalidValue;
-    const int RP = (RU + 15) / 16 * 16;
+    // rows padded to a multiple of 16; 65-80 rows run on the 96-row kernel (three
+    // 32-column warpgroups) rather than five 16-column ones at 768 threads
+    const int RP = RU > 64 ? 96 : (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess || p.all_slots) return e;  // a cascade call merges in the shared-prefix kernel
     return launch_programmatic(attn_combine_kernel, dim3((RU + COMBINE_ROWS - 1) / COMBINE_ROWS, p.units),

@@ -72,6 +72,13 @@ def test_attention_head_dim_64_and_no_gqa():
     check_full(a, "D=64, G=1")
 
 
+@pytest.mark.parametrize("D", [128, 64])
+def test_attention_80_rows_per_unit(D):
+    # N=16 x G=5 = 80 rows per KV head: one row chunk, padded to the 96-row kernel
+    a = W.make_attention_inputs(16, 10, 2, D, [700, 1500, 40, 2049], seed=38)
+    check_full(a, f"N=16, G=5, D={D}")
+
+
 def test_attention_many_rows_per_kv_head():
     # N=64 rows x G=4 -> 256 rows per KV head: two row chunks per unit
     a = W.make_attention_inputs(64, 8, 2, 128, [400, 64, 1200], seed=33, explicit_chain_mask=True)
