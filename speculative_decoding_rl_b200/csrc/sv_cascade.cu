@@ -177,6 +177,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
     uint64_t *o_full = p_empty + NP;  // [2] by tile parity: that tile's P V has completed
     uint64_t *q_ready = o_full + 2, *done_bar = q_ready + 1;
     uint64_t *pair_bar = done_bar + 1;  // [4] by lane quadrant: the two warps of a quadrant
+    // A two-slot K ring's slot of tile t is its S buffer t & 1, freed by the QK
+    // product s_full[t & 1] marks; two P buffers are freed by tile t's P V, which
+    // o_full[t & 1] marks: one commit fewer per tile each.
+    uint64_t *k_free = NK == 2 ? s_full : k_empty;
+    uint64_t *p_free = NP == 2 ? o_full : p_empty;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(base + L.off_misc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(base + L.off_misc + 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     const int blk = page * PAGE < P ? __ldg(bt + page) : -1;
                     blks[pg] = (blk >= 0 && blk < a.num_blocks) ? blk : a.num_blocks;  // past the pool: zeros
                 }
-                if (!mbar_wait(&k_empty[sk], kph ^ 1u, abort_flag, a.wait_limit_ns)) break;
+                if (!mbar_wait(&k_free[sk], kph ^ 1u, abort_flag, a.wait_limit_ns)) break;
                 mbar_arrive_expect_tx(&k_full[sk], L.tile);
                 uint8_t *kd = base + L.off_k + sk * L.tile;
 #pragma unroll
@@ -276,7 +281,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
         if (lane == 0 && ntiles > 0) {
             constexpr uint32_t ids = idesc_bf16(128, PF_KEYS, false, false);  // Q, K both K-major
             constexpr uint32_t idp = idesc_bf16(128, D, false, true);         // P K-major, V dims-major
-            const uint32_t qa = smem_u32(base + L.off_q);
+            // operand descriptors of the buffers; a product adds its stage's offset
+            // in 16-byte units (shared addresses stay below 2^18 bytes, so the
+            // 14-bit address field does not carry)
+            const uint64_t qdesc = sw128_desc(smem_u32(base + L.off_q), 16, 1024);
+            const uint64_t kdesc = sw128_desc(smem_u32(base + L.off_k), 16, 1024);
+            const uint64_t pdesc = sw128_desc(smem_u32(base + L.off_p), 16, 1024);
+            const uint64_t vdesc = sw128_desc(smem_u32(base + L.off_v), PF_ATOM, 1024);
             bool ok = mbar_wait(q_ready, 0, abort_flag, a.wait_limit_ns);
             int nq = 0, np = 0;
             int ks = 0, vs = 0, ps = 0;  // ring slots of tiles nq (K) and np (V, P) and their phases
@@ -289,15 +300,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     const int sk = ks, sb = nq & 1;
                     if (mbar_test(&k_full[sk], kph) && mbar_test(&s_empty[sb], ((nq >> 1) & 1) ^ 1)) {
                         tc_fence_after();
-                        const uint32_t ka = smem_u32(base + L.off_k + sk * L.tile);
+                        const uint64_t ka = kdesc + ((sk * L.tile) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(qa + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(ka + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
-                            mma_bf16_ss(tmem + COL_S + sb * PF_KEYS, ad, bd, ids, kk > 0);
+                            const uint32_t off = ((kk >> 2) * PF_ATOM + (kk & 3) * 32) >> 4;
+                            mma_bf16_ss(tmem + COL_S + sb * PF_KEYS, qdesc + off, ka + off, ids, kk > 0);
                         }
                         mma_commit(&s_full[sb]);
-                        mma_commit(&k_empty[sk]);
+                        if (NK != 2) mma_commit(&k_empty[sk]);
                         if (++ks == NK) { ks = 0; kph ^= 1u; }
                         ++nq;
                         progressed = true;
@@ -307,16 +317,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                     const int sv = vs, pb = ps;
                     if (mbar_test(&p_full[pb], pph) && mbar_test(&v_full[sv], vph)) {
                         tc_fence_after();
-                        const uint32_t va = smem_u32(base + L.off_v + sv * L.tile);
-                        const uint32_t pa = smem_u32(base + L.off_p + pb * 2 * PF_ATOM);
+                        const uint64_t va = vdesc + ((sv * L.tile) >> 4);
+                        const uint64_t pa = pdesc + ((pb * 2 * PF_ATOM) >> 4);
 #pragma unroll
                         for (int kk = 0; kk < PF_KEYS / 16; ++kk) {
-                            const uint64_t ad = sw128_desc(pa + (kk >> 2) * PF_ATOM + (kk & 3) * 32, 16, 1024);
-                            const uint64_t bd = sw128_desc(va + kk * 2048, PF_ATOM, 1024);
+                            const uint64_t ad = pa + (((kk >> 2) * PF_ATOM + (kk & 3) * 32) >> 4);
+                            const uint64_t bd = va + ((kk * 2048) >> 4);
                             mma_bf16_ss(tmem + COL_O, ad, bd, idp, (np > 0 || kk > 0) ? 1u : 0u);
                         }
                         mma_commit(&o_full[np & 1]);
-                        mma_commit(&p_empty[pb]);
+                        if (NP != 2) mma_commit(&p_empty[pb]);
                         mma_commit(&v_empty[sv]);
                         if (++vs == NV) { vs = 0; vph ^= 1u; }
                         if (++ps == NP) { ps = 0; pph ^= 1u; }
@@ -456,7 +466,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) cascade_prefix_kernel(const __g
                 tmem_wait_st();
             }
             m_run = m_new;
-            if (!(ok = wait_w(&p_empty[pb], pphase ^ 1u))) break;
+            if (!(ok = wait_w(&p_free[pb], pphase ^ 1u))) break;
             if (++pslot == NP) { pslot = 0; pphase ^= 1u; }
             uint8_t *pt = base + L.off_p + pb * 2 * PF_ATOM;
 #pragma unroll
