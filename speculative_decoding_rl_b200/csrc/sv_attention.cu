@@ -959,13 +959,23 @@ __global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const A
             acc.z = fmaf(w, ov[k].z, acc.z); acc.w = fmaf(w, ov[k].w, acc.w);
         }
     }
-    for (int k = COMBINE_REG_SEGS; k < n; ++k) {
-        const float w = k < 32 ? __shfl_sync(0xffffffffu, wl, k)
-                               : exp2f(__ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r) - M);
-        if (dl) {
-            const float4 o = __ldcg(reinterpret_cast<const float4 *>(seg0 + (size_t)k * sf + (size_t)r * D) + lane);
-            acc.x = fmaf(w, o.x, acc.x); acc.y = fmaf(w, o.y, acc.y);
-            acc.z = fmaf(w, o.z, acc.z); acc.w = fmaf(w, o.w, acc.w);
+    // the rest (a unit split over many CTAs, at small B) four at a time, the
+    // four loads in flight before the first is used
+    const size_t sf4 = sf / 4;  // slot stride in float4 (slots are 256-byte multiples)
+    const float4 *op = reinterpret_cast<const float4 *>(seg0 + (size_t)COMBINE_REG_SEGS * sf + (size_t)r * D) + lane;
+#pragma unroll 1
+    for (int k0 = COMBINE_REG_SEGS; k0 < n; k0 += 4, op += 4 * sf4) {
+        float4 ob[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            ob[j] = (k0 + j < n && dl) ? __ldcg(op + j * sf4) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int k = k0 + j;  // partials past n were loaded as zeros
+            const float w = k < 32 ? __shfl_sync(0xffffffffu, wl, k & 31)
+                                   : (k < n ? exp2f(__ldcg(seg0 + (size_t)k * sf + (size_t)RU * D + r) - M) : 0.f);
+            acc.x = fmaf(w, ob[j].x, acc.x); acc.y = fmaf(w, ob[j].y, acc.y);
+            acc.z = fmaf(w, ob[j].z, acc.z); acc.w = fmaf(w, ob[j].w, acc.w);
         }
     }
     if (!dl) return;
