@@ -894,7 +894,13 @@ SV_DEV int block_sum_i(int v, int *red) {
 // launch only after its own wait on earlier work: the schedule is recomputed
 // from ctx_lens (complete by then) before this kernel waits, so once the
 // attention kernel completes one round of loads remains.
-__global__ void __launch_bounds__(32 * COMBINE_ROWS) attn_combine_kernel(const AttnParams p) {
+// MIN_CTAS: CTAs per SM the register budget is sized for. Two when there are at
+// most a quarter as many units as attention CTAs (every unit is split about four
+// ways or more, and the extra registers keep more of its partials' loads in
+// flight); three otherwise (a unit has a few partials, and most of the
+// combine's CTAs return after the schedule test, so CTA turnover counts).
+template <int MIN_CTAS>
+__global__ void __launch_bounds__(32 * COMBINE_ROWS, MIN_CTAS) attn_combine_kernel(const AttnParams p) {
     griddep_launch_dependents();  // the next call's attention kernel may run its prologue
     const int u = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int D = p.D, RU = p.rows_unit;
@@ -1137,7 +1143,8 @@ cudaError_t launch_attention(const AttnParams &p, cudaStream_t stream) {
     const int RP = RU > 64 ? 96 : (RU + 15) / 16 * 16;
     cudaError_t e = p.D == 128 ? launch_tc_rp<128>(P, RP, stream) : launch_tc_rp<64>(P, RP, stream);
     if (e != cudaSuccess || p.all_slots) return e;  // a cascade call merges in the shared-prefix kernel
-    return launch_programmatic(attn_combine_kernel, dim3((RU + COMBINE_ROWS - 1) / COMBINE_ROWS, p.units),
+    return launch_programmatic(4 * p.units <= p.num_ctas ? attn_combine_kernel<2> : attn_combine_kernel<3>,
+                               dim3((RU + COMBINE_ROWS - 1) / COMBINE_ROWS, p.units),
                                dim3(32 * COMBINE_ROWS), 0, stream, p);
 }
 
